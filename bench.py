@@ -1,0 +1,418 @@
+"""Benchmark of the ConvRot linear on B200.
+
+One step = one pass of the whole online path (rotate + per-token quantize +
+integer GEMM + dequant) over every linear of the workload, for one batch of M
+synthetic tokens.  Default workload: the W8A8 ViT-L encoder linears (qkv
+1024->3072, proj 1024->1024, fc1 1024->4096, fc2 4096->1024) at M = 5184 tokens
+(72 x 72 patches), Hadamard block 128.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Multi-GPU runs (torchrun, one process per GPU) are independent replicas: each
+rank processes its own batch of tokens (M-split, no collective on the data
+path); the timed region is bracketed by barriers and the max over ranks counts.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rotated_bit_quantized_block_b200 import binding as cr  # noqa: E402
+from rotated_bit_quantized_block_b200 import workloads as wl  # noqa: E402
+
+METRIC = "ConvRot W8A8/W4A4 linear TOPS and tokens/s (rotate+quant+GEMM+dequant), % roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        self.out.flush()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.out.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ------------------------------------------------------------------------------------------ workload
+
+class Replica:
+    """Device buffers of one independent batch: per linear X, Y, codes, workspace."""
+
+    def __init__(self, w: wl.Workload, replica: int, device):
+        self.items = []
+        for i, lin in enumerate(w.linears):
+            X, W, _ = wl.linear_inputs(w, i, replica=replica)
+            Xd = torch.from_numpy(X).to(device)
+            Wd = torch.from_numpy(W).to(device)
+            Wq, sw = cr.convrot_quantize_weight(Wd, w.block, w.bits, cr.CLIP_MSE)
+            need = cr.convrot_workspace_bytes(w.M, lin.K, w.bits)
+            self.items.append({
+                "lin": lin, "X": Xd, "Xhost": torch.from_numpy(X).pin_memory(), "Wq": Wq, "sw": sw,
+                "Y": torch.empty((w.M, lin.N), dtype=torch.float16, device=device),
+                "Yhost": torch.empty((w.M, lin.N), dtype=torch.float16).pin_memory(),
+                "ws": torch.empty(need, dtype=torch.uint8, device=device),
+                "W": Wd,
+            })
+
+    def nbytes(self):
+        return sum(it["X"].nbytes + it["Y"].nbytes + it["Wq"].nbytes + it["ws"].nbytes for it in self.items)
+
+
+def run_step(w, rep, stream, gemm_events=None):
+    """One pass over every linear: rotate+quant kernel, then GEMM+dequant kernel.
+
+    The two kernels are launched through their own entry points (the same
+    launches convrot_linear_* makes) so that the GEMM can be bracketed by events.
+    """
+    for i, it in enumerate(rep.items):
+        lin = it["lin"]
+        ws = it["ws"]
+        code_bytes = w.M * lin.K * w.bits // 8
+        off = (code_bytes + 255) // 256 * 256
+        xq = ws[:code_bytes].view(torch.int8 if w.bits == 8 else torch.uint8).view(w.M, -1)
+        xs = ws[off:off + 4 * w.M].view(torch.float32)
+        cr.convrot_rotate_quant_act(it["X"], w.block, w.bits, Xq=xq, x_scale=xs, stream=stream)
+        if gemm_events is not None:
+            gemm_events[i][0].record(stream)
+        gemm = cr.convrot_gemm_w8a8 if w.bits == 8 else cr.convrot_gemm_w4a4
+        gemm(xq, xs, it["Wq"], it["sw"], Y=it["Y"], stream=stream)
+        if gemm_events is not None:
+            gemm_events[i][1].record(stream)
+
+
+def run_step_linear(w, rep, stream):
+    """One pass through the public linear entry point (what a user calls)."""
+    for it in rep.items:
+        fn = cr.convrot_linear_w8a8 if w.bits == 8 else cr.convrot_linear_w4a4
+        fn(it["X"], it["Wq"], it["sw"], w.block, None, it["Y"], it["ws"], stream)
+
+
+# ------------------------------------------------------------------------------------------ CPU oracle
+
+def time_oracle(w: wl.Workload, budget_s: float, max_rows: int | None = None):
+    """Times the CPU oracle (rotate+quant, integer GEMM, dequant) on a bounded
+    sample of rows of every linear of the workload.  The offline weight
+    conversion is done first and is not timed, as on the GPU."""
+    import oracle  # the oracle is only used by this baseline leg
+
+    threads = oracle.set_threads(os.cpu_count() or 1)
+    weights = []
+    for i in range(len(w.linears)):
+        X, W, _ = wl.linear_inputs(w, i)
+        qw, sw, _ = oracle.quantize_weight(W, w.block, w.bits, oracle.CLIP_MSE)
+        weights.append((X, qw, sw))
+
+    def run(rows):
+        t0 = time.perf_counter()
+        for X, qw, sw in weights:
+            oracle.linear(X[:rows], qw, sw, w.block, w.bits)
+        return time.perf_counter() - t0
+
+    rows = max(1, min(w.M, 2 * threads))
+    t = run(rows)
+    target = int(rows * budget_s / max(t, 1e-6))
+    rows = max(1, min(w.M if max_rows is None else max_rows, target))
+    t = run(rows)
+    return {"rows": rows, "seconds": t, "tokens_per_s": rows / t, "threads": threads,
+            "ops": sum(2 * rows * l.K * l.N for l in w.linears)}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ------------------------------------------------------------------------------------------ arms
+
+def reference_arm(args, w, rank, world):
+    """The oracle, as it stands, on the host cores: the CPU reference arm."""
+    if rank != 0:
+        return
+    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        time_oracle(w, budget / 4)
+    runs = [time_oracle(w, budget) for _ in range(args.steps)]
+    tps = [r["tokens_per_s"] for r in runs]
+    value = statistics.median(tps)
+    rows = runs[0]["rows"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * w.M / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8" if w.bits == 8 else "int4",
+        "data": "synthetic", "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": runs[0]["threads"], "kind": "oracle",
+                         "sample": f"{rows} of {w.M} tokens through every linear per step "
+                                   f"(rotate+quant, int GEMM, dequant); weights converted untimed; "
+                                   f"CPU {cpu_model()}"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "tops": value * sum(2 * l.K * l.N for l in w.linears) / 1e12,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w: wl.Workload):
+    return {
+        "workload": f"{w.name}: " + ", ".join(f"{l.name} {l.K}->{l.N}" for l in w.linears)
+                    + f"; M={w.M} tokens; Hadamard block {w.block}; W{w.bits}A{w.bits}; "
+                      f"acts N(0,1) with {w.outlier_frac:.1%} outlier channels x{w.outlier_factor:g}; "
+                      f"W N(0,{w.w_sigma})",
+        "M": w.M, "block": w.block, "bits": w.bits, "linears": [[l.name, l.K, l.N] for l in w.linears],
+        "parallelism": "replicas (M-split, no collective)",
+    }
+
+
+def ours_arm(args, w, rank, world, local_rank):
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    cr.load_library()
+    peaks = load_peaks()
+    stream = torch.cuda.Stream(device)
+
+    # offline conversion (timed once, reported separately; not part of a step)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    reps = [Replica(w, replica=rank * 2 + r, device=device) for r in range(2)]
+    torch.cuda.synchronize()
+    setup_s = time.perf_counter() - t0
+    per_set = reps[0].nbytes()
+    # offline weight conversion time, measured by itself
+    wq_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with torch.cuda.stream(stream):
+        wq_ev[0].record(stream)
+        for it in reps[0].items:
+            cr.convrot_quantize_weight(it["W"], w.block, w.bits, cr.CLIP_MSE, stream=stream)
+        wq_ev[1].record(stream)
+    torch.cuda.synchronize()
+    weight_quant_ms = wq_ev[0].elapsed_time(wq_ev[1])
+    for rep in reps:
+        for it in rep.items:
+            del it["W"]
+
+    # warm-up (eager), also initializes per-device kernel attributes before capture
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            run_step(w, reps[s % 2], stream)
+    torch.cuda.synchronize()
+    cr.convrot_device_status(stream)
+
+    # capture the K timed steps as one graph, with an event pair around every GEMM
+    n_lin = len(w.linears)
+    events = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(n_lin)]
+              for _ in range(args.steps)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for s in range(args.steps):
+            run_step(w, reps[s % 2], stream, gemm_events=events[s])
+    torch.cuda.synchronize()
+    graph.replay()  # one untimed replay of the captured steps
+    torch.cuda.synchronize()
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    gemm_ms = [[events[s][i][0].elapsed_time(events[s][i][1]) for i in range(n_lin)] for s in range(args.steps)]
+    cr.convrot_device_status(stream)
+    clocks = clk.summary()
+
+    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
+    elapsed_ms = float(t_max.item())
+    ms_per_step = elapsed_ms / args.steps
+    tokens = w.M * world * args.steps
+    value = tokens / (elapsed_ms / 1000.0)
+
+    # end to end through the public entry point, host buffers in pinned memory
+    h2d = sum(it["X"].nbytes for it in reps[0].items)
+    d2h = sum(it["Y"].nbytes for it in reps[0].items)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e_start.record(stream)
+        for s in range(args.steps):
+            rep = reps[s % 2]
+            for it in rep.items:
+                it["X"].copy_(it["Xhost"], non_blocking=True)
+            run_step_linear(w, rep, stream)
+            for it in rep.items:
+                it["Yhost"].copy_(it["Y"], non_blocking=True)
+        e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e_start.elapsed_time(e_end)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.barrier()
+    e2e_value = tokens / (float(e2e_ms.item()) / 1000.0)
+    cr.convrot_device_status(stream)
+
+    if rank != 0:
+        return
+    ops_step = w.ops()
+    gemm_total_ms = sum(sum(r) for r in gemm_ms)
+    gemm_ops_total = ops_step * args.steps
+    achieved_tops = gemm_ops_total / (gemm_total_ms / 1000.0) / 1e12
+    int8_peak = 2.0 * peaks["bf16_tflops"]  # dense int8 = 2 x dense bf16 (4.5 vs 2.25 POPS nominal)
+    per_linear_ms = [statistics.mean(gemm_ms[s][i] for s in range(args.steps)) for i in range(n_lin)]
+    act_ms_step = ms_per_step - sum(per_linear_ms)
+    act_bytes_step = sum(w.M * l.K * 2 + w.M * l.K * w.bits // 8 + 4 * w.M for l in w.linears)
+    roofline = {
+        "bound": "tensor", "achieved": achieved_tops, "peak": int8_peak, "unit": "TOPS",
+        "frac": achieved_tops / int8_peak, "traffic": None,
+        "kernel": "gemm_i8_tcgen05 (int8 x int8 -> int32, fused dequant epilogue)",
+        "peak_note": f"dense int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s",
+        "per_linear_ms": {l.name: round(t, 5) for l, t in zip(w.linears, per_linear_ms)},
+        "per_linear_tops": {l.name: round(2 * w.M * l.K * l.N / (t / 1000) / 1e12, 1)
+                            for l, t in zip(w.linears, per_linear_ms)},
+    }
+    act_gbs = act_bytes_step / (act_ms_step / 1000.0) / 1e9 if act_ms_step > 0 else None
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8" if w.bits == 8 else "int4 (int8 MMA)", "data": "synthetic",
+        "config": dict(config_of(w), l2=f"inputs larger than L2: 2 rotating buffer sets of "
+                                        f"{per_set / 2**20:.0f} MiB each (L2 {L2_BYTES >> 20} MiB)"),
+        "tops": ops_step * world * args.steps / (elapsed_ms / 1000.0) / 1e12,
+        "roofline": roofline,
+        "rotate_quant": {"bound": "hbm", "ms_per_step": act_ms_step, "achieved_gbs": act_gbs,
+                         "peak_gbs": peaks["hbm_gbs"],
+                         "frac": act_gbs / peaks["hbm_gbs"] if act_gbs else None,
+                         "note": "step time minus the GEMM launches (includes launch gaps)"},
+        "offline_weight_quant_ms": weight_quant_ms,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "convrot_linear_* with pinned-host X copied in and Y copied out every step"},
+        "gpu_launches": 2 * n_lin * args.steps,
+        "clocks": clocks,
+        "setup_s": setup_s,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        cb = time_oracle(w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {
+            "value": cb["tokens_per_s"], "unit": "tokens/s", "cores": cb["threads"], "kind": "oracle",
+            "sample": f"{cb['rows']} of {w.M} tokens through every linear (rotate+quant, int GEMM, dequant) "
+                      f"in {cb['seconds']:.1f} s; weights converted untimed; CPU {cpu_model()}",
+        }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="vit_l_w8a8")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.workload.startswith("msweep_M"):
+        w = wl.msweep(int(args.workload[len("msweep_M"):]))
+    else:
+        w = wl.WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, w, rank, world)
+        return
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        ours_arm(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,172 @@
+/*
+ * convrot.h -- C ABI of the ConvRot-quantized linear layer for NVIDIA B200
+ * (sm_100a).
+ *
+ * The method (source pages):
+ *   - civarchive.com, "SAM 3.1 Multiplex ConvRot" release, section
+ *     "Quantization recipe": an offline converter upcasts each eligible
+ *     linear weight to FP32, applies a block-Hadamard ConvRot transform,
+ *     chooses an MSE-optimized clipping scale and stores per-row scales;
+ *     the runtime performs W8A8 (or W4A4) operations with online, dynamic
+ *     per-operation activation quantization.  Section "Downloads": INT4
+ *     multiplication may fall back to INT8 multiplication where the hardware
+ *     has no INT4 path (sm_100 tcgen05 has none: int4 codes are widened to
+ *     int8 in shared memory ahead of the int8 MMA).
+ *   - trellis3d.app, "TRELLIS.2 INT8 ConvRot in ComfyUI", section "What
+ *     ConvRot changes": a grouped, normalized Hadamard rotation precedes the
+ *     per-row weight quantization and the matching rotation is applied to the
+ *     activations at runtime, spreading channel outliers over the grid.
+ *
+ * Notation.  X is M x K (tokens x in-features), W is N x K (out x in, as in
+ * nn.Linear), both row-major.  b ("block") is the Hadamard block size.
+ * R = blockdiag(H_b/sqrt(b), ...) with H_b the Sylvester Hadamard matrix.
+ *   X~ = X.R,  s_x[m] = max_k |X~[m,k]| / qmax,       qx = rne(X~ * (1/s_x))
+ *   W~ = W.R,  s_w[n] = alpha_n max_k |W~[n,k]| / qmax, qw = clamp(rne(W~ * (1/s_w)))
+ *   acc[m,n] = sum_k qx[m,k] qw[n,k]             (exact int32)
+ *   Y[m,n]   = fp16( (float(acc) * s_x[m]) * s_w[n] + bias[n] )
+ * qmax = 127 (int8, codes in [-127, 127]) or 7 (int4, codes in [-8, 7]).
+ * Rotation and scales are fp32; every rounding is round-to-nearest-even.
+ *
+ * Int4 storage: two codes per byte along K, element 2j in bits 0..3 and
+ * element 2j+1 in bits 4..7, 4-bit two's complement.  A packed row of K
+ * codes takes K/2 bytes.
+ *
+ * Conventions for every call below:
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     keeps no reference after the call returns.  Arrays are dense row-major.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and nothing synchronizes with the host, except
+ *     convrot_device_status().  Calls are safe to capture in a CUDA graph.
+ *   - Nothing is allocated; scratch space is the caller's `workspace`.
+ *   - Argument checks run before any launch.  On failure the call returns a
+ *     status other than CONVROT_OK, launches nothing and leaves every output
+ *     untouched; convrot_last_error() then describes the failure.
+ *   - Shape limits: 128 <= K <= 32768 with K % 128 == 0; b a power of two in
+ *     [1, 256] with K % b == 0; 0 <= M, N < 2^31 (M == 0 or N == 0 is a no-op);
+ *     the GEMM entry points need N % 8 == 0.  X, Y, Xq, Wq, workspace,
+ *     w_scale, bias and acc_out must be 16-byte aligned, x_scale 4-byte aligned.
+ *   - Non-finite inputs (inf / NaN in X or W) give unspecified codes.
+ *   - Kernels never trap: a device-side wait that exceeds its time limit
+ *     abandons the launch and records CONVROT_ERR_TIMEOUT, which
+ *     convrot_device_status() reports.
+ */
+#ifndef CONVROT_H
+#define CONVROT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CONVROT_OK = 0,
+    CONVROT_ERR_INVALID_ARG = 1, /* null pointer, bad enum, shape outside the limits */
+    CONVROT_ERR_UNSUPPORTED = 2, /* valid request this build does not handle (e.g. device not sm_100) */
+    CONVROT_ERR_ALIGNMENT = 3,   /* a pointer violates the alignment rules above */
+    CONVROT_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
+    CONVROT_ERR_TIMEOUT = 5,     /* a kernel abandoned a wait after its time limit */
+    CONVROT_ERR_WORKSPACE = 6    /* workspace null or smaller than convrot_workspace_bytes() */
+} convrot_status_t;
+
+enum { CONVROT_CLIP_ABSMAX = 0, CONVROT_CLIP_MSE = 1 };
+enum { CONVROT_DTYPE_F16 = 0, CONVROT_DTYPE_BF16 = 1, CONVROT_DTYPE_F32 = 2 };
+
+/*
+ * Offline weight conversion -- "Quantization recipe" steps 1-4 (civarchive
+ * ConvRot release page): upcast W to fp32, rotate each row by blockdiag(R_b),
+ * pick the per-row clip factor, store per-row scales and codes.
+ *   W        [N x K] source weight, element type w_dtype (fp16, bf16 or fp32).
+ *   clip_mode CONVROT_CLIP_ABSMAX: alpha = 1.  CONVROT_CLIP_MSE: alpha is the
+ *            first minimiser, scanning alpha = 1.00, 0.99, ..., 0.50, of the
+ *            float64 squared error sum_k (W~[n,k] - s*q)^2.
+ *   bits     8 -> Wq is int8 [N x K]; 4 -> Wq is packed int4 uint8 [N x K/2].
+ *   w_scale  [N] fp32 output, s_w[n] (0 for an all-zero row, whose codes are 0).
+ */
+convrot_status_t convrot_quantize_weight(const void *W, int w_dtype, int64_t N, int64_t K, int block,
+                                         int bits, int clip_mode, void *Wq, float *w_scale,
+                                         void *stream);
+
+/*
+ * Online activation quantization -- "online 8-bit activation quantization",
+ * "dynamic per-operation" (civarchive ConvRot release, "Quantization recipe"),
+ * with the matching rotation of "What ConvRot changes" (trellis3d.app):
+ * X~ = X.R in fp32, per-token absmax scale, round to nearest.
+ *   X        [M x K] fp16.
+ *   bits     8 -> Xq is int8 [M x K]; 4 -> Xq is packed int4 uint8 [M x K/2].
+ *   x_scale  [M] fp32 output, s_x[m] (0 for an all-zero row).
+ */
+convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, int block, int bits,
+                                          void *Xq, float *x_scale, void *stream);
+
+/*
+ * Bytes of scratch the linear entry points need for M tokens of K features:
+ * the activation codes (M*K for bits = 8, M*K/2 for bits = 4) and the M
+ * per-token scales, each rounded up to 256 bytes.  Returns 0 for invalid
+ * arguments.
+ */
+size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
+
+/*
+ * W8A8 ConvRot linear (civarchive ConvRot release, "The INT8 file uses W8A8
+ * operations"): Y = dequant( int8(rotate(X)) . Wq^T ) + bias.
+ *   X         [M x K] fp16 activations (not yet rotated).
+ *   Wq        [N x K] int8 codes from convrot_quantize_weight(bits = 8), same block.
+ *   w_scale   [N] fp32 per-output-row scales.
+ *   bias      [N] fp16 or NULL.
+ *   Y         [M x N] fp16 output.
+ *   workspace at least convrot_workspace_bytes(M, K, 8) bytes of device memory;
+ *             its contents on return are the activation codes and scales.
+ */
+convrot_status_t convrot_linear_w8a8(const void *X, int64_t M, int64_t K, const int8_t *Wq,
+                                     const float *w_scale, int64_t N, const void *bias, int block, void *Y,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * W4A4 ConvRot linear (civarchive ConvRot release, "The INT4 file similarly
+ * uses W4A4 operations"; INT8 multiplication on hardware without INT4 MMA).
+ * As convrot_linear_w8a8 with Wq the packed int4 codes [N x K/2] from
+ * convrot_quantize_weight(bits = 4) and workspace >=
+ * convrot_workspace_bytes(M, K, 4).
+ */
+convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const uint8_t *Wq,
+                                     const float *w_scale, int64_t N, const void *bias, int block, void *Y,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The integer GEMM with its dequantizing epilogue alone, on given codes (the
+ * last two steps of the linear): Y[m,n] = fp16((float(acc) * x_scale[m]) *
+ * w_scale[n] + bias[n]), acc = sum_k Xq[m,k] Wq[n,k].
+ *   Xq [M x K] int8, Wq [N x K] int8 (w8a8); packed int4 [M x K/2], [N x K/2] (w4a4).
+ *   acc_out  [M x N] int32 or NULL: receives acc (for exact-integer testing).
+ */
+convrot_status_t convrot_gemm_w8a8(const int8_t *Xq, const float *x_scale, int64_t M, const int8_t *Wq,
+                                   const float *w_scale, int64_t N, int64_t K, const void *bias, void *Y,
+                                   int32_t *acc_out, void *stream);
+convrot_status_t convrot_gemm_w4a4(const uint8_t *Xq, const float *x_scale, int64_t M, const uint8_t *Wq,
+                                   const float *w_scale, int64_t N, int64_t K, const void *bias, void *Y,
+                                   int32_t *acc_out, void *stream);
+
+/*
+ * Synchronizes `stream`, then returns and clears the sticky device-side
+ * status of the current device: CONVROT_OK, CONVROT_ERR_TIMEOUT if a kernel
+ * abandoned a wait since the last query, or CONVROT_ERR_CUDA if the stream
+ * reported an error.
+ */
+convrot_status_t convrot_device_status(void *stream);
+
+/* Static description of a status code (never NULL). */
+const char *convrot_status_string(convrot_status_t status);
+
+/* Detail of the most recent failing call on this host thread ("" if none). */
+const char *convrot_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int convrot_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONVROT_H */

@@ -1,0 +1,410 @@
+// convrot.cu -- the C ABI declared in include/convrot.h: argument validation,
+// TMA descriptor encoding and kernel launches.  One translation unit holds the
+// whole library so that the device status word has a single definition.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "../../include/convrot.h"
+#include "device_utils.cuh"
+#include "gemm_tcgen05.cuh"
+#include "rotate_quant.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+thread_local std::string g_last_error;
+
+convrot_status_t fail(convrot_status_t st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+convrot_status_t ok() { return CONVROT_OK; }
+
+#define CR_REQUIRE(cond, status, ...)                  \
+    do {                                               \
+        if (!(cond)) return fail(status, __VA_ARGS__); \
+    } while (0)
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+int ilog2(int64_t v) {
+    int l = 0;
+    while ((int64_t(1) << l) < v) ++l;
+    return l;
+}
+size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- device info
+
+struct DeviceInfo {
+    int major = 0, minor = 0, sms = 0;
+    bool attrs_set = false;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+convrot_status_t current_device(int *dev, DeviceInfo **info) {
+    cudaError_t e = cudaGetDevice(dev);
+    CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    CR_REQUIRE(*dev >= 0 && *dev < kMaxDevices, CONVROT_ERR_UNSUPPORTED, "device ordinal %d out of range", *dev);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo &d = g_dev[*dev];
+    if (d.sms == 0) {
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, *dev);
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, *dev);
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, *dev);
+        CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    }
+    *info = &d;
+    CR_REQUIRE(d.major == 10 && d.minor == 0, CONVROT_ERR_UNSUPPORTED,
+               "this library is built for sm_100a (B200); device %d is sm_%d%d", *dev, d.major, d.minor);
+    return ok();
+}
+
+convrot_status_t launch_status(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// A row-major byte matrix (rows x row_bytes) read in boxes of box_rows x
+// box_bytes.
+convrot_status_t make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t row_bytes, int box_rows,
+                          int box_bytes, bool swizzle128) {
+    EncodeTiledFn fn = encode_fn();
+    CR_REQUIRE(fn != nullptr, CONVROT_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CR_REQUIRE(r == CUDA_SUCCESS, CONVROT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return ok();
+}
+
+// ---------------------------------------------------------------- shared checks
+
+convrot_status_t check_shape(int64_t rows, int64_t K, int block, const char *rows_name) {
+    CR_REQUIRE(rows >= 0 && rows < (int64_t(1) << 31), CONVROT_ERR_INVALID_ARG, "%s = %lld out of [0, 2^31)",
+               rows_name, static_cast<long long>(rows));
+    CR_REQUIRE(K >= 128 && K <= 32768 && K % 128 == 0, CONVROT_ERR_INVALID_ARG,
+               "K = %lld must be a multiple of 128 in [128, 32768]", static_cast<long long>(K));
+    CR_REQUIRE(block >= 1 && block <= 256 && is_pow2(block) && K % block == 0, CONVROT_ERR_INVALID_ARG,
+               "block = %d must be a power of two in [1, 256] dividing K", block);
+    return ok();
+}
+
+convrot_status_t check_bits(int bits) {
+    CR_REQUIRE(bits == 8 || bits == 4, CONVROT_ERR_INVALID_ARG, "bits = %d must be 8 or 4", bits);
+    return ok();
+}
+
+#define CR_TRY(expr)                          \
+    do {                                      \
+        convrot_status_t st_ = (expr);        \
+        if (st_ != CONVROT_OK) return st_;    \
+    } while (0)
+
+// Rows per CTA and threads per CTA of the rotation kernels.
+void rotate_geometry(int64_t K, int *rows, int *threads) {
+    const int L = static_cast<int>(K / convrot::kElemsPerThread);
+    int R = L >= 256 ? 1 : 256 / L;
+    if (R > convrot::kMaxRowsPerCta) R = convrot::kMaxRowsPerCta;
+    *rows = R;
+    *threads = ((R * L + 31) / 32) * 32;
+}
+
+template <int LOG2B, int BITS>
+void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st) {
+    int R, T;
+    rotate_geometry(K, &R, &T);
+    const int64_t grid = (M + R - 1) / R;
+    convrot::act_rotate_quant_kernel<LOG2B, BITS><<<static_cast<unsigned>(grid), T, 0, st>>>(
+        static_cast<const __half *>(X), M, static_cast<int>(K), R, Xq, xs);
+}
+
+template <int BITS>
+void dispatch_act(int log2b, const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st) {
+    switch (log2b) {
+        case 0: launch_act<0, BITS>(X, M, K, Xq, xs, st); break;
+        case 1: launch_act<1, BITS>(X, M, K, Xq, xs, st); break;
+        case 2: launch_act<2, BITS>(X, M, K, Xq, xs, st); break;
+        case 3: launch_act<3, BITS>(X, M, K, Xq, xs, st); break;
+        case 4: launch_act<4, BITS>(X, M, K, Xq, xs, st); break;
+        case 5: launch_act<5, BITS>(X, M, K, Xq, xs, st); break;
+        case 6: launch_act<6, BITS>(X, M, K, Xq, xs, st); break;
+        case 7: launch_act<7, BITS>(X, M, K, Xq, xs, st); break;
+        default: launch_act<8, BITS>(X, M, K, Xq, xs, st); break;
+    }
+}
+
+template <int LOG2B>
+void launch_weight(const void *W, int dtype, int64_t N, int64_t K, int bits, int clip, void *Wq, float *ws,
+                   cudaStream_t st) {
+    int R, T;
+    rotate_geometry(K, &R, &T);
+    const int64_t grid = (N + R - 1) / R;
+    convrot::weight_rotate_quant_kernel<LOG2B><<<static_cast<unsigned>(grid), T, 0, st>>>(
+        W, dtype, N, static_cast<int>(K), R, bits, clip, Wq, ws);
+}
+
+convrot_status_t rotate_quant_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, void *Xq,
+                                       float *x_scale, cudaStream_t st) {
+    const int log2b = ilog2(block);
+    if (bits == 8) dispatch_act<8>(log2b, X, M, K, Xq, x_scale, st);
+    else dispatch_act<4>(log2b, X, M, K, Xq, x_scale, st);
+    return launch_status("act_rotate_quant");
+}
+
+// ---------------------------------------------------------------- GEMM launch
+
+template <class Cfg>
+convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *A, const void *B, int64_t M, int64_t N,
+                                 int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
+                                 int32_t *acc_out, cudaStream_t st) {
+    {
+        static std::mutex mu;
+        static bool done[kMaxDevices] = {};
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(convrot::gemm_i8_tcgen05_kernel<Cfg>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+            CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+            done[dev] = true;
+        }
+    }
+    CUtensorMap ta, tb;
+    const int64_t row_bytes = Cfg::W4 ? K / 2 : K;
+    const int box_bytes = Cfg::W4 ? Cfg::BK / 2 : Cfg::BK;
+    CR_TRY(make_map(&ta, A, M, row_bytes, Cfg::BM, box_bytes, !Cfg::W4));
+    CR_TRY(make_map(&tb, B, N, row_bytes, Cfg::BN, box_bytes, !Cfg::W4));
+    const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
+    const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
+    convrot::gemm_i8_tcgen05_kernel<Cfg><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, st>>>(
+        ta, tb, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sx, sw,
+        static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out);
+    return launch_status("gemm_i8_tcgen05");
+}
+
+// Picks the tile width: the widest tile that still gives every SM work.
+template <bool W4>
+convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *A, const void *B, int64_t M, int64_t N,
+                             int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
+                             int32_t *acc_out, cudaStream_t st) {
+    const int64_t tiles_m = (M + 127) / 128;
+    const int64_t tiles_256 = tiles_m * ((N + 255) / 256);
+    if (N >= 256 && tiles_256 >= info->sms)
+        return launch_gemm_cfg<convrot::GemmCfg<256, W4>>(info, dev, A, B, M, N, K, sx, sw, bias, Y, acc_out, st);
+    return launch_gemm_cfg<convrot::GemmCfg<128, W4>>(info, dev, A, B, M, N, K, sx, sw, bias, Y, acc_out, st);
+}
+
+convrot_status_t check_gemm_args(const void *Xq, const float *xs, int64_t M, const void *Wq, const float *ws,
+                                 int64_t N, int64_t K, const void *bias, const void *Y) {
+    CR_TRY(check_shape(M, K, 1, "M"));
+    CR_REQUIRE(N >= 0 && N < (int64_t(1) << 31), CONVROT_ERR_INVALID_ARG, "N = %lld out of [0, 2^31)",
+               static_cast<long long>(N));
+    CR_REQUIRE(N % 8 == 0, CONVROT_ERR_INVALID_ARG, "N = %lld must be a multiple of 8", static_cast<long long>(N));
+    if (M == 0 || N == 0) return ok();
+    CR_REQUIRE(Xq && xs && Wq && ws && Y, CONVROT_ERR_INVALID_ARG, "null pointer argument");
+    CR_REQUIRE(aligned(Xq, 16) && aligned(Wq, 16) && aligned(Y, 16), CONVROT_ERR_ALIGNMENT,
+               "codes and Y must be 16-byte aligned");
+    CR_REQUIRE(aligned(xs, 4), CONVROT_ERR_ALIGNMENT, "x_scale must be 4-byte aligned");
+    CR_REQUIRE(aligned(ws, 16), CONVROT_ERR_ALIGNMENT, "w_scale must be 16-byte aligned");
+    CR_REQUIRE(bias == nullptr || aligned(bias, 16), CONVROT_ERR_ALIGNMENT, "bias must be 16-byte aligned");
+    return ok();
+}
+
+}  // namespace
+
+// =============================================================================
+// C ABI
+// =============================================================================
+
+extern "C" {
+
+const char *convrot_status_string(convrot_status_t s) {
+    switch (s) {
+        case CONVROT_OK: return "ok";
+        case CONVROT_ERR_INVALID_ARG: return "invalid argument";
+        case CONVROT_ERR_UNSUPPORTED: return "unsupported";
+        case CONVROT_ERR_ALIGNMENT: return "misaligned pointer";
+        case CONVROT_ERR_CUDA: return "CUDA error";
+        case CONVROT_ERR_TIMEOUT: return "device wait timed out";
+        case CONVROT_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+const char *convrot_last_error(void) { return g_last_error.c_str(); }
+
+int convrot_version(void) { return kVersion; }
+
+size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits) {
+    if (M < 0 || K <= 0 || (bits != 8 && bits != 4)) return 0;
+    const size_t codes = static_cast<size_t>(M) * static_cast<size_t>(K) * static_cast<size_t>(bits) / 8;
+    return round256(codes) + round256(static_cast<size_t>(M) * 4);
+}
+
+convrot_status_t convrot_quantize_weight(const void *W, int w_dtype, int64_t N, int64_t K, int block, int bits,
+                                         int clip_mode, void *Wq, float *w_scale, void *stream) {
+    g_last_error.clear();
+    CR_TRY(check_shape(N, K, block, "N"));
+    CR_TRY(check_bits(bits));
+    CR_REQUIRE(w_dtype >= CONVROT_DTYPE_F16 && w_dtype <= CONVROT_DTYPE_F32, CONVROT_ERR_INVALID_ARG,
+               "w_dtype = %d is not one of fp16 / bf16 / fp32", w_dtype);
+    CR_REQUIRE(clip_mode == CONVROT_CLIP_ABSMAX || clip_mode == CONVROT_CLIP_MSE, CONVROT_ERR_INVALID_ARG,
+               "clip_mode = %d", clip_mode);
+    if (N == 0) return ok();
+    CR_REQUIRE(W && Wq && w_scale, CONVROT_ERR_INVALID_ARG, "null pointer argument");
+    CR_REQUIRE(aligned(W, 16) && aligned(Wq, 16), CONVROT_ERR_ALIGNMENT, "W and Wq must be 16-byte aligned");
+    CR_REQUIRE(aligned(w_scale, 4), CONVROT_ERR_ALIGNMENT, "w_scale must be 4-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (ilog2(block)) {
+        case 0: launch_weight<0>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
+        case 1: launch_weight<1>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
+        case 2: launch_weight<2>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
+        case 3: launch_weight<3>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
+        case 4: launch_weight<4>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
+        case 5: launch_weight<5>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
+        case 6: launch_weight<6>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
+        case 7: launch_weight<7>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
+        default: launch_weight<8>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
+    }
+    return launch_status("weight_rotate_quant");
+}
+
+convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, int block, int bits, void *Xq,
+                                          float *x_scale, void *stream) {
+    g_last_error.clear();
+    CR_TRY(check_shape(M, K, block, "M"));
+    CR_TRY(check_bits(bits));
+    if (M == 0) return ok();
+    CR_REQUIRE(X && Xq && x_scale, CONVROT_ERR_INVALID_ARG, "null pointer argument");
+    CR_REQUIRE(aligned(X, 16) && aligned(Xq, 16), CONVROT_ERR_ALIGNMENT, "X and Xq must be 16-byte aligned");
+    CR_REQUIRE(aligned(x_scale, 4), CONVROT_ERR_ALIGNMENT, "x_scale must be 4-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    return rotate_quant_act_impl(X, M, K, block, bits, Xq, x_scale, static_cast<cudaStream_t>(stream));
+}
+
+static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t K, const void *Wq,
+                                    const float *w_scale, int64_t N, const void *bias, int block, void *Y,
+                                    void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    CR_TRY(check_shape(M, K, block, "M"));
+    CR_REQUIRE(N >= 0 && N < (int64_t(1) << 31) && N % 8 == 0, CONVROT_ERR_INVALID_ARG,
+               "N = %lld must be a multiple of 8 in [0, 2^31)", static_cast<long long>(N));
+    if (M == 0 || N == 0) return ok();
+    CR_REQUIRE(X && Wq && w_scale && Y, CONVROT_ERR_INVALID_ARG, "null pointer argument");
+    const size_t need = convrot_workspace_bytes(M, K, bits);
+    CR_REQUIRE(workspace != nullptr && workspace_bytes >= need, CONVROT_ERR_WORKSPACE,
+               "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+    CR_REQUIRE(aligned(workspace, 16), CONVROT_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+    CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *xq = ws;
+    float *xs = reinterpret_cast<float *>(ws + round256(static_cast<size_t>(M) * K * bits / 8));
+    CR_TRY(check_gemm_args(xq, xs, M, Wq, w_scale, N, K, bias, Y));
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CR_TRY(rotate_quant_act_impl(X, M, K, block, bits, xq, xs, st));
+    if (bits == 8) return launch_gemm<false>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
+    return launch_gemm<true>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
+}
+
+convrot_status_t convrot_linear_w8a8(const void *X, int64_t M, int64_t K, const int8_t *Wq, const float *w_scale,
+                                     int64_t N, const void *bias, int block, void *Y, void *workspace,
+                                     size_t workspace_bytes, void *stream) {
+    return linear_impl(8, X, M, K, Wq, w_scale, N, bias, block, Y, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const uint8_t *Wq, const float *w_scale,
+                                     int64_t N, const void *bias, int block, void *Y, void *workspace,
+                                     size_t workspace_bytes, void *stream) {
+    return linear_impl(4, X, M, K, Wq, w_scale, N, bias, block, Y, workspace, workspace_bytes, stream);
+}
+
+static convrot_status_t gemm_impl(bool w4, const void *Xq, const float *x_scale, int64_t M, const void *Wq,
+                                  const float *w_scale, int64_t N, int64_t K, const void *bias, void *Y,
+                                  int32_t *acc_out, void *stream) {
+    g_last_error.clear();
+    CR_TRY(check_gemm_args(Xq, x_scale, M, Wq, w_scale, N, K, bias, Y));
+    if (M == 0 || N == 0) return ok();
+    CR_REQUIRE(acc_out == nullptr || aligned(acc_out, 16), CONVROT_ERR_ALIGNMENT, "acc_out must be 16-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (w4) return launch_gemm<true>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st);
+    return launch_gemm<false>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st);
+}
+
+convrot_status_t convrot_gemm_w8a8(const int8_t *Xq, const float *x_scale, int64_t M, const int8_t *Wq,
+                                   const float *w_scale, int64_t N, int64_t K, const void *bias, void *Y,
+                                   int32_t *acc_out, void *stream) {
+    return gemm_impl(false, Xq, x_scale, M, Wq, w_scale, N, K, bias, Y, acc_out, stream);
+}
+
+convrot_status_t convrot_gemm_w4a4(const uint8_t *Xq, const float *x_scale, int64_t M, const uint8_t *Wq,
+                                   const float *w_scale, int64_t N, int64_t K, const void *bias, void *Y,
+                                   int32_t *acc_out, void *stream) {
+    return gemm_impl(true, Xq, x_scale, M, Wq, w_scale, N, K, bias, Y, acc_out, stream);
+}
+
+convrot_status_t convrot_device_status(void *stream) {
+    g_last_error.clear();
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+    unsigned int word = 0;
+    e = cudaMemcpyFromSymbol(&word, convrot::g_device_status, sizeof(word));
+    CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (word != 0) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(convrot::g_device_status, &zero, sizeof(zero));
+        if (word & convrot::kStatusTimeout)
+            return fail(CONVROT_ERR_TIMEOUT, "a kernel abandoned a device-side wait (status 0x%x)", word);
+    }
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,315 @@
+// gemm_tcgen05.cuh -- integer GEMM with the dequantizing epilogue of the
+// ConvRot linear, on sm_100a 5th-generation tensor cores.
+//
+//   acc[m,n] = sum_k qx[m,k] * qw[n,k]                      (tcgen05.mma kind::i8, int32 in TMEM)
+//   Y[m,n]   = fp16( (float(acc) * s_x[m]) * s_w[n] + bias[n] )   (fused epilogue)
+//
+// Method: civarchive.com "SAM 3.1 Multiplex ConvRot" release, "Quantization
+// recipe" (W8A8 / W4A4 operations, per-row scales; INT4 multiplication falls
+// back to INT8 multiplication where the hardware has no INT4 path -- sm_100
+// tcgen05 has no integer-4 kind, so W4A4 tiles are widened to int8 in shared
+// memory before the int8 MMA).
+//
+// Structure: persistent, warp-specialized CTAs (one per SM), output tile
+// 128 x BN, K step 128 bytes.
+//   warp 0      TMA producer (one elected lane): A and B tiles -> smem ring
+//   warp 1      TMEM allocator + MMA issuer (one lane): 4 x tcgen05.mma per K step
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, fp16, store
+//   warps 6-9   (W4A4 only) nibble -> byte converters between a packed ring
+//               and the MMA ring
+// Two TMEM accumulators (2 x BN columns) let the epilogue of one tile overlap
+// the main loop of the next.  No TMA multicast is used anywhere.
+#pragma once
+
+#include "device_utils.cuh"
+
+namespace convrot {
+
+template <int BN_, bool W4_>
+struct GemmCfg {
+    static constexpr int BM = 128;
+    static constexpr int BN = BN_;
+    static constexpr int BK = 128;  // K elements per stage (= bytes of one int8 row segment)
+    static constexpr bool W4 = W4_;
+    static constexpr int A_BYTES = BM * BK;
+    static constexpr int B_BYTES = BN * BK;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    // MMA ring depth and (W4A4) packed ring depth
+    static constexpr int STAGES = W4 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 4 : 6);
+    static constexpr int PSTAGES = W4 ? (BN == 256 ? 3 : 4) : 0;
+    static constexpr int PA_BYTES = A_BYTES / 2;
+    static constexpr int PB_BYTES = B_BYTES / 2;
+    static constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int NUM_THREADS = W4 ? 320 : 192;
+    static constexpr int NUM_BARRIERS = 2 * STAGES + 2 * PSTAGES + 4 + 1;
+    static constexpr int SMEM_BYTES =
+        1024 /* alignment slack */ + STAGES * STAGE_BYTES + PSTAGES * PSTAGE_BYTES + NUM_BARRIERS * 8 + 16;
+    static constexpr uint32_t IDESC = idesc_i8(BM, BN);
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
+};
+
+// Bounded wait used while draining: ignores the abort flag, still time-limited.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
+    int dummy = 0;
+    mbar_wait(bar, parity, &dummy);
+}
+
+// Sign-extends 16 packed int4 codes (8 bytes, low nibble = even element) to 16
+// bytes holding 16 * code: shifting each nibble into the high half of its byte
+// keeps the sign; the products are rescaled by 1/256 in the epilogue.
+__device__ __forceinline__ uint4 widen_int4x16(uint2 p) {
+    const uint32_t lo0 = (p.x << 4) & 0xf0f0f0f0u, hi0 = p.x & 0xf0f0f0f0u;
+    const uint32_t lo1 = (p.y << 4) & 0xf0f0f0f0u, hi1 = p.y & 0xf0f0f0f0u;
+    return make_uint4(__byte_perm(lo0, hi0, 0x5140), __byte_perm(lo0, hi0, 0x7362), __byte_perm(lo1, hi1, 0x5140),
+                      __byte_perm(lo1, hi1, 0x7362));
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
+    gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                           int N, int K, const float *__restrict__ sx, const float *__restrict__ sw,
+                           const __half *__restrict__ bias, __half *__restrict__ Y, int32_t *__restrict__ acc_out) {
+    constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, PSTAGES = Cfg::PSTAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ring = smem;                                          // STAGES x (A | B), int8, 128B-swizzled
+    uint8_t *pring = ring + STAGES * Cfg::STAGE_BYTES;             // PSTAGES x (A4 | B4), packed, dense rows
+    uint64_t *bars = reinterpret_cast<uint64_t *>(pring + PSTAGES * Cfg::PSTAGE_BYTES);
+    uint64_t *full = bars;                                         // MMA ring: operands ready
+    uint64_t *empty = full + STAGES;                               // MMA ring: slot consumed
+    uint64_t *pfull = empty + STAGES;                              // packed ring: TMA landed
+    uint64_t *pempty = pfull + PSTAGES;                            // packed ring: slot converted
+    uint64_t *tmem_full = pempty + PSTAGES;                        // [2] accumulator ready
+    uint64_t *tmem_empty = tmem_full + 2;                          // [2] accumulator drained
+    uint64_t *drain = tmem_empty + 2;                              // MMA completion at exit
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
+    const int num_tiles = tiles_m * tiles_n;
+    const int num_kb = K / Cfg::BK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&full[i], Cfg::W4 ? 128 : 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < PSTAGES; ++i) {
+            mbar_init(&pfull[i], 1);
+            mbar_init(&pempty[i], 128);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tmem_full[i], 1);
+            mbar_init(&tmem_empty[i], 128);
+        }
+        mbar_init(drain, 1);
+        *abort = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const int nst = Cfg::W4 ? PSTAGES : STAGES;
+            uint64_t *ld_full = Cfg::W4 ? pfull : full;
+            uint64_t *ld_empty = Cfg::W4 ? pempty : empty;
+            uint32_t last_parity[(Cfg::W4 ? PSTAGES : STAGES)];
+            bool filled[(Cfg::W4 ? PSTAGES : STAGES)];
+            for (int i = 0; i < nst; ++i) filled[i] = false;
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&ld_empty[s], ph ^ 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (Cfg::W4) {
+                        uint8_t *dst = pring + s * Cfg::PSTAGE_BYTES;
+                        mbar_arrive_expect_tx(&ld_full[s], Cfg::PSTAGE_BYTES);
+                        tma_load_2d(dst, &tmA, &ld_full[s], kb * (Cfg::BK / 2), tm * BM);
+                        tma_load_2d(dst + Cfg::PA_BYTES, &tmB, &ld_full[s], kb * (Cfg::BK / 2), tn * BN);
+                    } else {
+                        uint8_t *dst = ring + s * Cfg::STAGE_BYTES;
+                        mbar_arrive_expect_tx(&ld_full[s], Cfg::STAGE_BYTES);
+                        tma_load_2d(dst, &tmA, &ld_full[s], kb * Cfg::BK, tm * BM);
+                        tma_load_2d(dst + Cfg::A_BYTES, &tmB, &ld_full[s], kb * Cfg::BK, tn * BN);
+                    }
+                    filled[s] = true;
+                    last_parity[s] = ph;
+                    if (++s == nst) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+            }
+            // no bulk copy may still be writing shared memory when the CTA exits
+            for (int i = 0; i < nst; ++i)
+                if (filled[i]) mbar_wait_drain(&ld_full[i], last_parity[i]);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            int local = 0;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++local) {
+                const int acc = local & 1;
+                const uint32_t acc_ph = (local >> 1) & 1;
+                if (!mbar_wait(&tmem_empty[acc], acc_ph ^ 1, abort)) break;
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&full[s], ph, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_addr(ring + s * Cfg::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + Cfg::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < Cfg::BK / 32; ++kk) {
+                        umma_i8(d_tmem, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
+                                Cfg::IDESC, (kb | kk) != 0);
+                    }
+                    umma_commit(&empty[s]);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (ok) umma_commit(&tmem_full[acc]);
+            }
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            const int acc = local & 1;
+            const uint32_t acc_ph = (local >> 1) & 1;
+            if (!mbar_wait(&tmem_full[acc], acc_ph, abort)) break;
+            tc_fence_after_sync();
+            const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
+            const int row = tm * BM + q * 32 + lane;
+            const bool row_ok = row < M;
+            const float sxm = row_ok ? sx[row] : 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                __syncwarp();  // tcgen05.ld is warp-collective
+                uint32_t r[32];
+                tmem_ld_32x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, r);
+                tmem_ld_wait();
+                const int col0 = tn * BN + c * 32;
+                if (!row_ok || col0 >= N) continue;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {  // 8 columns per 16-byte store
+                    const int col = col0 + 8 * g;
+                    if (col >= N) break;
+                    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(sw + col));
+                    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(sw + col + 4));
+                    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    float bv[8];
+                    if (bias != nullptr) {
+                        const uint4 braw = __ldg(reinterpret_cast<const uint4 *>(bias + col));
+                        const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&bw[i]));
+                            bv[2 * i] = p.x;
+                            bv[2 * i + 1] = p.y;
+                        }
+                    }
+                    int32_t av[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int32_t raw = static_cast<int32_t>(r[8 * g + i]);
+                        av[i] = Cfg::W4 ? (raw >> 8) : raw;  // W4A4 operands carry 16 * code each
+                    }
+                    uint32_t out[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float2 t = make_float2(__int2float_rn(av[2 * i]), __int2float_rn(av[2 * i + 1]));
+                        t = __fmul2_rn(t, make_float2(sxm, sxm));
+                        t = __fmul2_rn(t, make_float2(wv[2 * i], wv[2 * i + 1]));
+                        if (bias != nullptr) t = __fadd2_rn(t, make_float2(bv[2 * i], bv[2 * i + 1]));
+                        const __half2 h = __floats2half2_rn(t.x, t.y);
+                        out[i] = *reinterpret_cast<const uint32_t *>(&h);
+                    }
+                    *reinterpret_cast<uint4 *>(Y + static_cast<int64_t>(row) * N + col) =
+                        make_uint4(out[0], out[1], out[2], out[3]);
+                    if (acc_out != nullptr) {
+                        int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col);
+                        dst[0] = make_int4(av[0], av[1], av[2], av[3]);
+                        dst[1] = make_int4(av[4], av[5], av[6], av[7]);
+                    }
+                }
+            }
+            __syncwarp();
+            tc_fence_before_sync();
+            mbar_arrive(&tmem_empty[acc]);
+        }
+    } else if (Cfg::W4) {
+        // ------------------------------------------------------------ int4 -> int8 converters
+        const int ct = threadIdx.x - 192;  // 0..127
+        int ps = 0, us = 0;
+        uint32_t pph = 0, uph = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!mbar_wait(&pfull[ps], pph, abort) || !mbar_wait(&empty[us], uph ^ 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *src = pring + ps * Cfg::PSTAGE_BYTES;
+                uint8_t *dst = ring + us * Cfg::STAGE_BYTES;
+                constexpr int PIECES = (BM + BN) * (Cfg::BK / 16);  // 16 codes per piece
+#pragma unroll 4
+                for (int idx = ct; idx < PIECES; idx += 128) {
+                    const int rr = idx >> 3, piece = idx & 7;  // row over A then B; 16-byte chunk in the row
+                    const uint2 p = *reinterpret_cast<const uint2 *>(src + rr * 64 + piece * 8);
+                    *reinterpret_cast<uint4 *>(dst + rr * 128 + ((piece ^ (rr & 7)) << 4)) = widen_int4x16(p);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&full[us]);
+                mbar_arrive(&pempty[ps]);
+                if (++ps == PSTAGES) {
+                    ps = 0;
+                    pph ^= 1;
+                }
+                if (++us == STAGES) {
+                    us = 0;
+                    uph ^= 1;
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace convrot

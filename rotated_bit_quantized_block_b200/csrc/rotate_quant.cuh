@@ -1,0 +1,387 @@
+// rotate_quant.cuh -- block-Hadamard rotation fused with symmetric per-row
+// quantization, for activations (online, per token) and weights (offline,
+// per output row, with the MSE clip search).
+//
+// Method: civarchive.com "SAM 3.1 Multiplex ConvRot" release, "Quantization
+// recipe" (block-Hadamard ConvRot transform, per-row scales, online dynamic
+// activation quantization); trellis3d.app "TRELLIS.2 INT8 ConvRot",
+// "What ConvRot changes" (grouped, normalized Hadamard rotation of weights and
+// the matching rotation of activations).
+//
+// Register layout.  A row of K elements is split into 128-element groups;
+// four consecutive threads own one group, each holding 32 elements as four
+// 16-byte chunks: thread l of the row (g = l / 4, p = l % 4) holds, for chunk
+// j in 0..3 and e in 0..7, element 128*g + 8*p + 32*j + e.  Index bits 0-2
+// (e) and 5-6 (j) are butterflied in registers, bits 3 and 4 (p) between lanes
+// l^1 and l^2, and bit 7 (g's low bit, blocks of 256) between lanes l^4.  The
+// values are kept as float2 pairs (chunk h, chunk h + 2) so that every stage
+// but the one on bit 6 runs on the packed fp32x2 pipe.
+#pragma once
+
+#include "device_utils.cuh"
+
+namespace convrot {
+
+constexpr int kThreadsPerRowGroup = 4;  // threads per 128 elements
+constexpr int kElemsPerThread = 32;
+constexpr int kMaxRowsPerCta = 64;       // 256 threads / 4 threads per row (K = 128)
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer (RNE)
+
+// fp32(1 / sqrt(2^L)), L = 0..8 (correctly rounded decimal literals).
+__device__ __forceinline__ float rsqrt_block(int log2b) {
+    switch (log2b) {
+        case 0: return 1.0f;
+        case 1: return 0.70710678118654752440f;
+        case 2: return 0.5f;
+        case 3: return 0.35355339059327376220f;
+        case 4: return 0.25f;
+        case 5: return 0.17677669529663688110f;
+        case 6: return 0.125f;
+        case 7: return 0.088388347648318440550f;
+        default: return 0.0625f;
+    }
+}
+
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// a - b on the packed pipe (b * -1 is exact, so this is one rounding).
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, f2(-1.0f), a); }
+
+// One butterfly stage between lanes `lane` and `lane ^ m`: the lower lane keeps
+// a + b, the upper one a - b (a = lower lane's value, b = upper lane's).
+__device__ __forceinline__ void lane_stage(float2 (&v)[2][8], int lane, int m) {
+    const float sgn = (lane & m) ? -1.0f : 1.0f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float2 other;
+            other.x = __shfl_xor_sync(0xffffffffu, v[h][e].x, m);
+            other.y = __shfl_xor_sync(0xffffffffu, v[h][e].y, m);
+            v[h][e] = __ffma2_rn(v[h][e], f2(sgn), other);
+        }
+    }
+}
+
+// Unnormalized Walsh-Hadamard transform (Sylvester order) of every block of
+// 2^LOG2B elements held by the thread group (see the layout above).
+template <int LOG2B>
+__device__ __forceinline__ void fwht_block(float2 (&v)[2][8], int lane) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        if (k < LOG2B) {
+            const int m = 1 << k;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (!(e & m)) {
+                        const float2 a = v[h][e], b = v[h][e | m];
+                        v[h][e] = __fadd2_rn(a, b);
+                        v[h][e | m] = sub2(a, b);
+                    }
+                }
+            }
+        }
+    }
+    if (LOG2B > 3) lane_stage(v, lane, 1);
+    if (LOG2B > 4) lane_stage(v, lane, 2);
+    if (LOG2B > 5) {  // bit 5: chunk pairs (0,1) and (2,3) -> h = 0 vs h = 1
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float2 a = v[0][e], b = v[1][e];
+            v[0][e] = __fadd2_rn(a, b);
+            v[1][e] = sub2(a, b);
+        }
+    }
+    if (LOG2B > 6) {  // bit 6: chunk j vs j + 2 -> inside each float2
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float a = v[h][e].x, b = v[h][e].y;
+                v[h][e] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+            }
+        }
+    }
+    if (LOG2B > 7) lane_stage(v, lane, 4);
+}
+
+// Loads the thread's 32 source elements of one row and upcasts them to fp32.
+// dtype: 0 fp16, 1 bf16, 2 fp32.  `elem0` = 128*g + 8*p.
+__device__ __forceinline__ void load_row_chunks(const void *row_base, int dtype, int elem0, float2 (&v)[2][8]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float f[8];
+        if (dtype == 2) {
+            const float *src = static_cast<const float *>(row_base) + elem0 + 32 * j;
+            const uint4 a = ld_stream_v4(src), b = ld_stream_v4(src + 4);
+            f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y);
+            f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+            f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y);
+            f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+        } else {
+            const uint16_t *src = static_cast<const uint16_t *>(row_base) + elem0 + 32 * j;
+            const uint4 a = ld_stream_v4(src);
+            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (dtype == 0) {
+                    const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+                    f[2 * i] = p.x;
+                    f[2 * i + 1] = p.y;
+                } else {
+                    f[2 * i] = __uint_as_float(w[i] << 16);
+                    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (j < 2) v[j][e].x = f[e];
+            else v[j - 2][e].y = f[e];
+        }
+    }
+}
+
+__device__ __forceinline__ float chunk_val(const float2 (&v)[2][8], int j, int e) {
+    return j < 2 ? v[j][e].x : v[j - 2][e].y;
+}
+
+// Low byte of the bit pattern of (t + 1.5*2^23): rne(t) in 8-bit two's complement.
+__device__ __forceinline__ uint32_t code_bits(const float2 (&r)[2][8], int j, int e) {
+    return __float_as_uint(chunk_val(r, j, e));
+}
+
+// Packs the 8 codes of chunk j (low bytes of `r`) as int8: two 32-bit words.
+__device__ __forceinline__ uint2 pack_int8_chunk(const float2 (&r)[2][8], int j) {
+    const uint32_t a = __byte_perm(code_bits(r, j, 0), code_bits(r, j, 1), 0x0040);
+    const uint32_t b = __byte_perm(code_bits(r, j, 2), code_bits(r, j, 3), 0x0040);
+    const uint32_t c = __byte_perm(code_bits(r, j, 4), code_bits(r, j, 5), 0x0040);
+    const uint32_t d = __byte_perm(code_bits(r, j, 6), code_bits(r, j, 7), 0x0040);
+    return make_uint2(__byte_perm(a, b, 0x5410), __byte_perm(c, d, 0x5410));
+}
+
+// Packs the 8 codes of chunk j as int4: byte i = code[2i] | code[2i+1] << 4.
+__device__ __forceinline__ uint32_t pack_int4_chunk(const float2 (&r)[2][8], int j) {
+    const uint32_t e02 = __byte_perm(code_bits(r, j, 0), code_bits(r, j, 2), 0x0040);
+    const uint32_t e46 = __byte_perm(code_bits(r, j, 4), code_bits(r, j, 6), 0x0040);
+    const uint32_t e13 = __byte_perm(code_bits(r, j, 1), code_bits(r, j, 3), 0x0040);
+    const uint32_t e57 = __byte_perm(code_bits(r, j, 5), code_bits(r, j, 7), 0x0040);
+    const uint32_t even = __byte_perm(e02, e46, 0x5410);
+    const uint32_t odd = __byte_perm(e13, e57, 0x5410);
+    return (even & 0x0f0f0f0fu) | ((odd & 0x0f0f0f0fu) << 4);
+}
+
+// Stores the thread's 32 codes (already in the low bytes of `r`).
+template <int BITS>
+__device__ __forceinline__ void store_codes(void *out_row, int elem0, const float2 (&r)[2][8]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (BITS == 8) {
+            *reinterpret_cast<uint2 *>(static_cast<int8_t *>(out_row) + elem0 + 32 * j) = pack_int8_chunk(r, j);
+        } else {
+            *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(out_row) + (elem0 + 32 * j) / 2) =
+                pack_int4_chunk(r, j);
+        }
+    }
+}
+
+// Largest power of two dividing L, at most 32: the lanes of one row that a
+// shuffle reduction may combine.
+__host__ __device__ __forceinline__ int reduce_width(int L) {
+    int g = L & (-L);
+    return g > 32 ? 32 : g;
+}
+
+// ---------------------------------------------------------------------------
+// Online activation path: X (fp16, M x K) -> codes + per-token scales.
+// One CTA handles `rows` consecutive rows with L = K/32 threads each; the
+// block is padded to a multiple of 32 threads (padding threads only join the
+// shuffles and barriers).
+// ---------------------------------------------------------------------------
+template <int LOG2B, int BITS>
+__global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__restrict__ X, int64_t M, int K,
+                                                                int rows, void *__restrict__ Xq,
+                                                                float *__restrict__ x_scale) {
+    __shared__ unsigned int s_amax[kMaxRowsPerCta];
+    __shared__ float s_inv[kMaxRowsPerCta];
+    const int L = K / kElemsPerThread;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int r = tid / L;
+    const int l = tid - r * L;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * rows + r;
+    const bool active = (r < rows) && (row < M);
+    const int elem0 = 128 * (l >> 2) + 8 * (l & 3);
+    constexpr float qmax = BITS == 8 ? 127.0f : 7.0f;
+
+    float2 v[2][8];
+    if (active) {
+        load_row_chunks(X + row * K, 0, elem0, v);
+    } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[h][e] = f2(0.0f);
+    }
+    if (tid < rows) s_amax[tid] = 0u;
+    __syncthreads();
+
+    fwht_block<LOG2B>(v, lane);
+    const float2 rb = f2(rsqrt_block(LOG2B));
+    float amax = 0.0f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            v[h][e] = __fmul2_rn(v[h][e], rb);
+            amax = fmaxf(amax, fmaxf(fabsf(v[h][e].x), fabsf(v[h][e].y)));
+        }
+    }
+    const int G = reduce_width(L);
+    for (int m = 1; m < G; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    if (r < rows && (l & (G - 1)) == 0) atomicMax(&s_amax[r], __float_as_uint(amax));  // amax >= 0
+    __syncthreads();
+    if (active && l == 0) {
+        const float s = __fdiv_rn(__uint_as_float(s_amax[r]), qmax);
+        s_inv[r] = s == 0.0f ? 0.0f : __frcp_rn(s);
+        x_scale[row] = s;
+    }
+    __syncthreads();
+    if (!active) return;
+    const float2 inv = f2(s_inv[r]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[h][e] = __fadd2_rn(__fmul2_rn(v[h][e], inv), f2(kRoundMagic));
+    void *out_row = BITS == 8 ? static_cast<void *>(static_cast<int8_t *>(Xq) + row * K)
+                              : static_cast<void *>(static_cast<uint8_t *>(Xq) + row * (K / 2));
+    store_codes<BITS>(out_row, elem0, v);
+}
+
+// ---------------------------------------------------------------------------
+// Offline weight path: W (fp16/bf16/fp32, N x K) -> fp32 -> rotation ->
+// per-row clip search -> codes + per-row scales.  Same thread layout as the
+// activation kernel.  The squared errors are reduced in a fixed order
+// (lanes, then row segments in index order), so the choice is deterministic.
+// ---------------------------------------------------------------------------
+constexpr int kMseGrid = 51;
+
+template <int LOG2B>
+__global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *__restrict__ W, int dtype,
+                                                                   int64_t N, int K, int rows, int bits,
+                                                                   int clip_mode, void *__restrict__ Wq,
+                                                                   float *__restrict__ w_scale) {
+    __shared__ unsigned int s_amax[kMaxRowsPerCta];
+    __shared__ float s_scale[kMaxRowsPerCta][kMseGrid];
+    __shared__ double s_part[256];  // one partial sum per (row, segment of G lanes): at most 1024 / 4
+    __shared__ double s_best_err[kMaxRowsPerCta];
+    __shared__ int s_best[kMaxRowsPerCta];
+    const int L = K / kElemsPerThread;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int r = tid / L;
+    const int l = tid - r * L;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * rows + r;
+    const bool active = (r < rows) && (row < N);
+    const int elem0 = 128 * (l >> 2) + 8 * (l & 3);
+    const int qmax = bits == 8 ? 127 : 7;
+    const int qmin = bits == 8 ? -127 : -8;
+    const int G = reduce_width(L);
+    const int segs = L / G;
+
+    float2 v[2][8];
+    if (active) {
+        const size_t esize = dtype == 2 ? 4 : 2;
+        load_row_chunks(static_cast<const char *>(W) + row * K * esize, dtype, elem0, v);
+    } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[h][e] = f2(0.0f);
+    }
+    if (tid < rows) {
+        s_amax[tid] = 0u;
+        s_best[tid] = 0;
+        s_best_err[tid] = __longlong_as_double(0x7ff0000000000000ll);  // +inf
+    }
+    __syncthreads();
+    fwht_block<LOG2B>(v, lane);
+    const float2 rb = f2(rsqrt_block(LOG2B));
+    float amax = 0.0f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            v[h][e] = __fmul2_rn(v[h][e], rb);
+            amax = fmaxf(amax, fmaxf(fabsf(v[h][e].x), fabsf(v[h][e].y)));
+        }
+    }
+    for (int m = 1; m < G; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    if (r < rows && (l & (G - 1)) == 0) atomicMax(&s_amax[r], __float_as_uint(amax));
+    __syncthreads();
+    const int n_alpha = clip_mode == 1 ? kMseGrid : 1;
+    // grid point i: alpha = fp32((100 - i) / 100), s = fp32(fp32(alpha * amax) / qmax)
+    if (r < rows) {
+        for (int i = l; i < n_alpha; i += L) {
+            const float alpha = __fdiv_rn(static_cast<float>(100 - i), 100.0f);
+            s_scale[r][i] = __fdiv_rn(__fmul_rn(alpha, __uint_as_float(s_amax[r])), static_cast<float>(qmax));
+        }
+    }
+    __syncthreads();
+    if (n_alpha > 1) {
+        for (int i = 0; i < n_alpha; ++i) {
+            const float s = r < rows ? s_scale[r][i] : 0.0f;
+            const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
+            const double sd = static_cast<double>(s);
+            double err = 0.0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float xs[2] = {v[h][e].x, v[h][e].y};
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const float t = __fmul_rn(xs[c], inv);
+                        const float q = fminf(fmaxf(rintf(t), static_cast<float>(qmin)), static_cast<float>(qmax));
+                        const double d = fma(-sd, static_cast<double>(q), static_cast<double>(xs[c]));
+                        err = fma(d, d, err);
+                    }
+                }
+            }
+            for (int m = 1; m < G; m <<= 1) err += __shfl_xor_sync(0xffffffffu, err, m);
+            if (r < rows && (l & (G - 1)) == 0) s_part[r * segs + l / G] = err;
+            __syncthreads();
+            if (r < rows && l == 0) {
+                double tot = 0.0;
+                for (int sgi = 0; sgi < segs; ++sgi) tot += s_part[r * segs + sgi];
+                if (tot < s_best_err[r]) {
+                    s_best_err[r] = tot;
+                    s_best[r] = i;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (!active) return;
+    const float s = s_scale[r][s_best[r]];
+    const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
+    if (l == 0) w_scale[row] = s;
+    float2 q[2][8];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float a = fminf(fmaxf(rintf(__fmul_rn(v[h][e].x, inv)), static_cast<float>(qmin)), static_cast<float>(qmax));
+            float b = fminf(fmaxf(rintf(__fmul_rn(v[h][e].y, inv)), static_cast<float>(qmin)), static_cast<float>(qmax));
+            // re-encode the (exact, small) integers with the rounding magic so
+            // that the packers can take their low bytes
+            q[h][e] = make_float2(__fadd_rn(a, kRoundMagic), __fadd_rn(b, kRoundMagic));
+        }
+    }
+    if (bits == 8) store_codes<8>(static_cast<int8_t *>(Wq) + row * K, elem0, q);
+    else store_codes<4>(static_cast<uint8_t *>(Wq) + row * (K / 2), elem0, q);
+}
+
+}  // namespace convrot

@@ -1,0 +1,296 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bars (from the method's statement of the problem):
+  * integer codes from the rotation kernels: within 1 code on at most 0.1 % of
+    elements (the GPU rotates with an fp32 butterfly, the oracle rounds an fp64
+    product), bit-exact where the butterfly is exact;
+  * int32 accumulators and fp16 outputs of the GEMM given identical codes and
+    scales: bit-exact;
+  * the whole linear: relative Frobenius error <= 2e-3 against the oracle.
+Inputs are seeded synthetic tensors from ``workloads`` with the shapes and
+outlier statistics of the benchmarked configurations.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from rotated_bit_quantized_block_b200 import binding as cr
+from rotated_bit_quantized_block_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+CODE_FRAC = 1e-3
+REL_FRO = 2e-3
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def unpack(q, bits):
+    return oracle.unpack_int4(q) if bits == 4 else q
+
+
+def assert_codes_close(got, ref, frac=CODE_FRAC):
+    d = np.abs(got.astype(np.int32) - ref.astype(np.int32))
+    assert d.max(initial=0) <= 1, f"code difference {d.max()}"
+    assert np.count_nonzero(d) <= frac * d.size, f"{np.count_nonzero(d)} of {d.size} codes differ"
+
+
+def rel_fro(a, b):
+    a = a.astype(np.float64)
+    b = b.astype(np.float64)
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
+
+
+@pytest.fixture(autouse=True)
+def _status_clean():
+    yield
+    cr.convrot_device_status()
+
+
+def gpu_act(X, b, bits):
+    Xq, s = cr.convrot_rotate_quant_act(dev(X), b, bits)
+    return unpack(host(Xq), bits), host(s)
+
+
+# ----------------------------------------------------------------------------- activations
+
+ACT_CASES = [
+    (64, 256, 64, 8), (64, 256, 64, 4),          # the tiny configuration
+    (1, 128, 128, 8), (7, 384, 128, 4), (65, 1536, 128, 8), (300, 6144, 128, 4),
+    (33, 1024, 256, 8), (130, 4096, 32, 4), (3, 32768, 256, 8), (129, 128, 1, 8),
+]
+
+
+@pytest.mark.parametrize("M,K,b,bits", ACT_CASES)
+def test_act_rotate_quant_matches_oracle(M, K, b, bits):
+    X = wl.activations(M, K, 0.01, 30.0, seed=M * 7 + K)
+    q, s = gpu_act(X, b, bits)
+    qr, sr = oracle.rotate_quant_act(X, b, bits)
+    assert np.allclose(s, sr, rtol=1e-5, atol=0)
+    assert_codes_close(q, qr)
+
+
+@pytest.mark.parametrize("b", [1, 2, 4, 8, 16, 32, 64, 128, 256])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_act_every_block_size(b, bits):
+    X = wl.activations(37, 1024, 0.02, 20.0, seed=b + bits)
+    q, s = gpu_act(X, b, bits)
+    qr, sr = oracle.rotate_quant_act(X, b, bits)
+    assert np.allclose(s, sr, rtol=1e-5, atol=0)
+    assert_codes_close(q, qr)
+
+
+@pytest.mark.parametrize("b", [1, 4, 16, 64, 256])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_act_bit_exact_when_butterfly_is_exact(b, bits):
+    """Small-integer inputs and b a power of 4 make every butterfly sum and the
+    1/sqrt(b) factor exact in fp32, so codes and scales must match bit for bit."""
+    rng = np.random.default_rng(b)
+    X = rng.integers(-8, 9, size=(70, 1024)).astype(np.float16)
+    X[5] = 0  # an all-zero token
+    q, s = gpu_act(X, b, bits)
+    qr, sr = oracle.rotate_quant_act(X, b, bits)
+    assert np.array_equal(s.view(np.uint32), sr.view(np.uint32))
+    assert np.array_equal(q, qr)
+    assert s[5] == 0 and np.all(q[5] == 0)
+
+
+@pytest.mark.parametrize("name,idx", [("vit_l_w8a8", 0), ("vit_l_w8a8", 3), ("vit_l_w4a4", 3), ("dit_w8a8", 2)])
+def test_act_full_size_sampled_rows(name, idx):
+    w = wl.WORKLOADS[name]
+    X, _, _ = wl.linear_inputs(w, idx)
+    q, s = gpu_act(X, w.block, w.bits)
+    rows = np.unique(np.concatenate([[0, 1, w.M - 1], np.linspace(0, w.M - 1, 61).astype(int)]))
+    qr, sr = oracle.rotate_quant_act(X[rows], w.block, w.bits)
+    assert np.allclose(s[rows], sr, rtol=1e-5, atol=0)
+    assert_codes_close(q[rows], qr)
+
+
+# ----------------------------------------------------------------------------- weights
+
+def gpu_weight(W, b, bits, clip, dtype=torch.float16):
+    Wt = dev(W) if dtype == torch.float16 else dev(W.astype(np.float32)).to(dtype)
+    Wq, s = cr.convrot_quantize_weight(Wt, b, bits, clip)
+    return unpack(host(Wq), bits), host(s)
+
+
+@pytest.mark.parametrize("N,K,b,bits", [(256, 256, 64, 8), (24, 384, 128, 4), (72, 1024, 128, 8),
+                                        (8, 6144, 256, 4), (100, 1536, 16, 8)])
+def test_weight_absmax_matches_oracle(N, K, b, bits):
+    W = wl.weight(N, K, 0.02, seed=N + K)
+    q, s = gpu_weight(W, b, bits, cr.CLIP_ABSMAX)
+    qr, sr, _ = oracle.quantize_weight(W, b, bits, oracle.CLIP_ABSMAX)
+    assert np.allclose(s, sr, rtol=1e-5, atol=0)
+    assert_codes_close(q, qr)
+
+
+def _check_mse_rows(W, b, bits, q, s, dtype=oracle.DTYPE_F16, Wsrc=None):
+    src = W if Wsrc is None else Wsrc
+    qr, sr, aidx, errs = oracle.quantize_weight(src, b, bits, oracle.CLIP_MSE, dtype=dtype, want_errs=True)
+    if dtype == oracle.DTYPE_F32:
+        x64 = src.astype(np.float64)
+    elif dtype == oracle.DTYPE_BF16:
+        x64 = oracle.decode(src, oracle.DTYPE_BF16)
+    else:
+        x64 = src.astype(np.float64)
+    _, w32 = oracle.rotate(x64, b)
+    same = np.isclose(s, sr, rtol=1e-5, atol=0)
+    # rows whose clip choice differs must be near-ties under the oracle's own error
+    for n in np.nonzero(~same)[0]:
+        e_gpu = oracle.quant_error(w32[n], s[n], bits)
+        best = errs[n, aidx[n]]
+        assert e_gpu <= best * (1 + 1e-5) + 1e-30, (n, e_gpu, best)
+    assert np.count_nonzero(~same) <= max(1, 0.02 * len(s))
+    assert_codes_close(q[same], qr[same])
+
+
+@pytest.mark.parametrize("N,K,b,bits", [(256, 256, 64, 8), (64, 1024, 128, 4), (48, 4096, 128, 8),
+                                        (16, 6144, 128, 4), (33, 512, 8, 4)])
+def test_weight_mse_clip_matches_oracle(N, K, b, bits):
+    W = wl.weight(N, K, 0.02, seed=3 * N + K)
+    # heavy-tailed rows so that the clip search has real decisions to make
+    W[::3] = (np.random.default_rng(N).standard_t(3, size=W[::3].shape) * 0.02).astype(np.float16)
+    q, s = gpu_weight(W, b, bits, cr.CLIP_MSE)
+    _check_mse_rows(W, b, bits, q, s)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_weight_source_dtypes(dtype):
+    rng = np.random.default_rng(0)
+    W32 = (rng.standard_normal((40, 512)) * 0.02).astype(np.float32)
+    Wt = dev(W32).to(dtype)
+    Wq, s = cr.convrot_quantize_weight(Wt, 128, 8, cr.CLIP_MSE)
+    q, s = host(Wq), host(s)
+    if dtype == torch.float32:
+        _check_mse_rows(None, 128, 8, q, s, oracle.DTYPE_F32, Wsrc=W32)
+    else:
+        bits16 = Wt.view(torch.int16).cpu().numpy().view(np.uint16)
+        _check_mse_rows(None, 128, 8, q, s, oracle.DTYPE_BF16, Wsrc=bits16)
+
+
+# ----------------------------------------------------------------------------- GEMM (bit-exact)
+
+def oracle_codes(M, N, K, b, bits, seed, full_range=False):
+    if full_range:
+        rng = np.random.default_rng(seed)
+        lo, hi = (-127, 128) if bits == 8 else (-8, 8)
+        qx = rng.integers(lo, hi, size=(M, K)).astype(np.int8)
+        qw = rng.integers(lo, hi, size=(N, K)).astype(np.int8)
+        sx = (rng.random(M) * 0.01 + 1e-4).astype(np.float32)
+        sw = (rng.random(N) * 0.01 + 1e-4).astype(np.float32)
+        return qx, sx, qw, sw
+    X = wl.activations(M, K, 0.01, 30.0, seed)
+    W = wl.weight(N, K, 0.02, seed + 1)
+    qx, sx = oracle.rotate_quant_act(X, b, bits)
+    qw, sw, _ = oracle.quantize_weight(W, b, bits, oracle.CLIP_MSE)
+    return qx, sx, qw, sw
+
+
+def run_gemm(qx, sx, qw, sw, bias, bits):
+    if bits == 8:
+        args = (dev(qx), dev(sx), dev(qw), dev(sw))
+        fn = cr.convrot_gemm_w8a8
+    else:
+        args = (dev(oracle.pack_int4(qx)), dev(sx), dev(oracle.pack_int4(qw)), dev(sw))
+        fn = cr.convrot_gemm_w4a4
+    acc = torch.empty((qx.shape[0], qw.shape[0]), dtype=torch.int32, device="cuda")
+    y = fn(*args, bias=None if bias is None else dev(bias), acc_out=acc)
+    return host(y), host(acc)
+
+
+GEMM_CASES = [
+    (64, 256, 256), (1, 8, 128), (7, 24, 384), (130, 264, 640), (300, 1000, 1024),
+    (256, 512, 4096), (129, 3072, 1024), (1000, 1536, 6144), (517, 4096, 256),
+]
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("M,N,K", GEMM_CASES)
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_gemm_bit_exact(M, N, K, bits, with_bias):
+    qx, sx, qw, sw = oracle_codes(M, N, K, 128, bits, seed=M + N + K)
+    bias = wl.bias(N, seed=N) if with_bias else None
+    y, acc = run_gemm(qx, sx, qw, sw, bias, bits)
+    yr, accr = oracle.gemm_dequant(qx, sx, qw, sw, bias, want_acc=True)
+    assert np.array_equal(acc, accr)
+    assert np.array_equal(y.view(np.uint16), yr.view(np.uint16))
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("M,N,K", [(200, 512, 2048), (64, 256, 32768)])
+def test_gemm_bit_exact_full_code_range(M, N, K, bits):
+    qx, sx, qw, sw = oracle_codes(M, N, K, 128, bits, seed=K, full_range=True)
+    y, acc = run_gemm(qx, sx, qw, sw, None, bits)
+    yr, accr = oracle.gemm_dequant(qx, sx, qw, sw, None, want_acc=True)
+    assert np.array_equal(acc, accr)
+    assert np.array_equal(y.view(np.uint16), yr.view(np.uint16))
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_gemm_full_size_sampled_rows(bits):
+    """ViT-L fc1 shape at full M; the oracle recomputes a sample of rows."""
+    M, N, K = 5184, 4096, 1024
+    qx, sx, qw, sw = oracle_codes(M, N, K, 128, bits, seed=11)
+    y, acc = run_gemm(qx, sx, qw, sw, None, bits)
+    rows = np.unique(np.concatenate([[0, 127, 128, M - 1], np.linspace(0, M - 1, 40).astype(int)]))
+    yr, accr = oracle.gemm_dequant(qx[rows], sx[rows], qw, sw, None, want_acc=True)
+    assert np.array_equal(acc[rows], accr)
+    assert np.array_equal(y[rows].view(np.uint16), yr.view(np.uint16))
+
+
+# ----------------------------------------------------------------------------- whole linear
+
+def linear_pair(w, idx, M=None, with_bias=False, sample=None):
+    X, W, bias = wl.linear_inputs(w, idx, M=M, with_bias=with_bias)
+    lin = cr.QuantizedLinear(dev(W), None if bias is None else dev(bias), w.block, w.bits, cr.CLIP_MSE)
+    y = host(lin(dev(X)))
+    qw, sw, _ = oracle.quantize_weight(W, w.block, w.bits, oracle.CLIP_MSE)
+    rows = np.arange(X.shape[0]) if sample is None else sample
+    yr = oracle.linear(X[rows], qw, sw, w.block, w.bits, bias)
+    ref = X[rows].astype(np.float64) @ W.astype(np.float64).T
+    if bias is not None:
+        ref += bias.astype(np.float64)
+    return y[rows], yr, ref
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_linear_tiny_config(bits):
+    w = wl.WORKLOADS["tiny_w8a8"]
+    w = wl.Workload(w.name, w.M, w.linears, bits, w.block, w.outlier_frac, w.outlier_factor, w.w_sigma, w.seed)
+    y, yr, ref = linear_pair(w, 0, with_bias=True)
+    assert rel_fro(y, yr) <= REL_FRO
+    assert rel_fro(y, ref) <= (0.02 if bits == 8 else 0.3)
+
+
+@pytest.mark.parametrize("name", ["vit_l_w8a8", "vit_l_w4a4"])
+@pytest.mark.parametrize("idx", [0, 1, 2, 3])
+def test_linear_vit_full_size_sampled(name, idx):
+    w = wl.WORKLOADS[name]
+    rows = np.unique(np.concatenate([[0, w.M - 1], np.linspace(0, w.M - 1, 48).astype(int)]))
+    y, yr, ref = linear_pair(w, idx, sample=rows)
+    assert rel_fro(y, yr) <= REL_FRO
+    assert rel_fro(y, ref) <= (0.02 if w.bits == 8 else 0.3)
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2])
+def test_linear_dit_full_size_sampled(idx):
+    w = wl.WORKLOADS["dit_w8a8"]
+    rows = np.linspace(0, w.M - 1, 24).astype(int)
+    y, yr, _ = linear_pair(w, idx, sample=rows)
+    assert rel_fro(y, yr) <= REL_FRO
+
+
+@pytest.mark.parametrize("M", wl.MSWEEP_M)
+def test_linear_msweep(M):
+    w = wl.msweep(M)
+    rows = None if M <= 128 else np.linspace(0, M - 1, 24).astype(int)
+    y, yr, _ = linear_pair(w, 0, sample=rows)
+    assert rel_fro(y, yr) <= REL_FRO
