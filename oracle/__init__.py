@@ -86,6 +86,7 @@ def _load():
         "oracle_unpack_int4": (i32, [P, i64, P]),
         "oracle_weight_bytes": (i64, [i64, i64, i32]),
         "oracle_gemm_dequant": (i32, [P, P, i64, P, P, i64, i64, P, P, P]),
+        "oracle_epilogue_value": (f32, [i32, f32, f32, f32]),
         "oracle_set_threads": (i32, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -250,7 +251,7 @@ def weight_bytes(N: int, K: int, bits: int) -> int:
 # ----------------------------------------------------------------------------
 
 def gemm_dequant(qx, sx, qw, sw, bias_f16=None, want_acc: bool = False):
-    """y = fp16(((float)acc * s_x[m]) * s_w[n] + bias[n]), acc = qx . qw^T (int).
+    """y = fp16(fma(fp32((float)acc * s_x[m]), s_w[n], bias[n])), acc = qx . qw^T (int).
 
     Codes are unpacked int8 (int4 values simply lie in [-8, 7]).  Returns y as
     np.float16 (M x N) and, if asked, the int32 accumulators.
@@ -274,6 +275,16 @@ def gemm_dequant(qx, sx, qw, sw, bias_f16=None, want_acc: bool = False):
                                        _ptr(acc), _ptr(y)), "gemm_dequant")
     y = y.view(np.float16)
     return (y, acc) if want_acc else y
+
+
+def epilogue_value(acc: int, sx: float, sw: float, bias: float) -> float:
+    """fp32 value of one output before the fp16 conversion: fma(fp32(acc * sx), sw, bias)."""
+    return _load().oracle_epilogue_value(int(acc), float(sx), float(sw), float(bias))
+
+
+def quantize_value(x: float, inv: float, bits: int) -> int:
+    """clamp(rne(x * inv)) with the exact product."""
+    return _load().oracle_quantize_value(float(x), float(inv), bits)
 
 
 def linear(X_f16, w_codes, w_scales, b: int, bits: int, bias_f16=None):

@@ -30,11 +30,13 @@
  *            alpha in {100/100, 99/100, ..., 50/100} for the MSE clip search
  *            (first strict minimum of the fp64 squared error, largest alpha
  *            first, so a tie keeps the larger alpha).
- *   q      = clamp( rne( fp32( x * fp32(1/s) ) ), qmin, qmax ),
+ *   q      = clamp( rne( x * fp32(1/s) ), qmin, qmax ), the product taken
+ *            exactly (one rounding, to the integer grid; ties to even),
  *            int8: [-127, 127], int4: [-8, 7].  s == 0 gives q == 0.
  *   int4   : two codes per byte, element 2j in bits 0..3, 2j+1 in bits 4..7.
  *   acc    = sum_k qx[m,k] * qw[n,k]   (exact integer, must fit int32)
- *   y      = fp16_rne( fp32( fp32( fp32(float(acc) * s_x[m]) * s_w[n] ) + bias[n] ) )
+ *   y      = fp16_rne( fma_fp32( fp32(float(acc) * s_x[m]), s_w[n], bias[n] ) ),
+ *            the last multiply-add rounded once (bias 0 when absent)
  *
  * Compile with -ffp-contract=off so that no multiply-add is fused.
  */
@@ -219,12 +221,14 @@ float oracle_scale(float amax, float alpha, int bits)
 /* fp32(1/s); a zero scale maps every value to code 0. */
 float oracle_inv_scale(float s) { return s == 0.0f ? 0.0f : 1.0f / s; }
 
-/* q = clamp(rne(fp32(x * inv)), qmin, qmax) */
+/* q = clamp(rne(x * inv), qmin, qmax) with the product exact: two 24-bit
+ * significands multiply exactly in float64, and nearbyint rounds that exact
+ * value to the nearest integer, ties to even. */
 int oracle_quantize_value(float x, float inv, int bits)
 {
-    float t = x * inv;
-    float r = nearbyintf(t); /* default rounding mode: nearest, ties to even */
-    float lo = (float)oracle_qmin(bits), hi = (float)oracle_qmax(bits);
+    double t = (double)x * (double)inv;
+    double r = nearbyint(t); /* default rounding mode: nearest, ties to even */
+    double lo = (double)oracle_qmin(bits), hi = (double)oracle_qmax(bits);
     if (r < lo) r = lo;
     if (r > hi) r = hi;
     return (int)r;
@@ -397,12 +401,19 @@ int oracle_gemm_dequant(const int8_t *qx, const float *sx, int64_t M, const int8
             if (acc_out) acc_out[m * N + n] = (int32_t)acc;
             float f = (float)(int32_t)acc;
             float t = f * sx[m];
-            t = t * sw[n];
-            if (bias) t = t + (float)oracle_f16_to_f64(bias[n]);
-            y[m * N + n] = oracle_f32_to_f16(t);
+            float b = bias ? (float)oracle_f16_to_f64(bias[n]) : 0.0f;
+            y[m * N + n] = oracle_f32_to_f16(fmaf(t, sw[n], b)); /* C99 fmaf: one rounding */
         }
     }
     return overflow ? ORACLE_ERR_OVERFLOW : ORACLE_OK;
+}
+
+/* fp32 value of one output before its fp16 conversion (for pinning the
+ * single-rounding multiply-add). */
+float oracle_epilogue_value(int32_t acc, float sx, float sw, float bias)
+{
+    float t = (float)acc * sx;
+    return fmaf(t, sw, bias);
 }
 
 int oracle_set_threads(int n)

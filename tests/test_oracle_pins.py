@@ -382,3 +382,60 @@ def test_end_to_end_error_bound(bits, b):
     assert np.all(np.abs(y - ref) <= bound)
     rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
     assert rel < (0.5 if bits == 4 else 0.02 if b > 1 else 0.05)
+
+
+# ---------------------------------------------------------------- single roundings, checked exactly
+
+def _nearest_int_even(fr):
+    """Nearest integer to a Fraction, ties to even."""
+    from fractions import Fraction
+    f = fr.numerator // fr.denominator
+    rem = fr - f
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and f % 2 == 1):
+        f += 1
+    return f
+
+
+def _is_nearest_f32(exact, r32):
+    """r32 is the float32 nearest to the Fraction `exact` (ties to even mantissa)."""
+    from fractions import Fraction
+    r = np.float32(r32)
+    lo = np.nextafter(r, np.float32(-np.inf))
+    hi = np.nextafter(r, np.float32(np.inf))
+    d = abs(Fraction(float(r)) - exact)
+    for nb in (lo, hi):
+        dn = abs(Fraction(float(nb)) - exact)
+        if dn < d:
+            return False
+        if dn == d and (int(r.view(np.uint32)) & 1):
+            return False
+    return True
+
+
+def test_quantizer_rounds_the_exact_product_once():
+    from fractions import Fraction
+    rng = np.random.default_rng(21)
+    xs = (rng.standard_normal(3000) * 20).astype(np.float32)
+    invs = (rng.random(3000) * 10 + 0.01).astype(np.float32)
+    # plus the half-way cases where fp32(x * inv) lands on k + 0.5
+    xs = np.concatenate([xs, np.float32([9.0, 6.25, 1.25, 7.75, -7.375])])
+    invs = np.concatenate([invs, np.float32([7.0555553, 0.4, 0.4, 8.193548, 8.610169])])
+    for x, inv in zip(xs, invs):
+        ref = _nearest_int_even(Fraction(float(x)) * Fraction(float(inv)))
+        ref = max(-127, min(127, ref))
+        assert oracle.quantize_value(x, inv, 8) == ref, (x, inv)
+    assert oracle.quantize_value(np.float32(9.0), np.float32(7.0555553), 8) == 63  # fp32(x*inv) would say 63.5 -> 64
+
+
+def test_epilogue_multiply_add_rounds_once():
+    from fractions import Fraction
+    rng = np.random.default_rng(22)
+    for _ in range(3000):
+        acc = int(rng.integers(-2**24, 2**24))
+        sx = np.float32(rng.random() * 0.1)
+        sw = np.float32(rng.random() * 0.01)
+        bias = np.float32(np.float16(rng.standard_normal() * 0.05))
+        got = np.float32(oracle.epilogue_value(acc, sx, sw, bias))
+        t = np.float32(np.float32(acc) * sx)  # IEEE fp32 product
+        exact = Fraction(float(t)) * Fraction(float(sw)) + Fraction(float(bias))
+        assert _is_nearest_f32(exact, got), (acc, sx, sw, bias)
