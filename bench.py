@@ -279,14 +279,15 @@ def ours_arm(args, w, rank, world, local_rank):
         for s in range(args.steps):
             run_step(w, reps[s % 2], stream, gemm_events=events[s])
     torch.cuda.synchronize()
-    graph.replay()  # one untimed replay of the captured steps
+    with torch.cuda.stream(stream):
+        graph.replay()  # one untimed replay of the captured steps
     torch.cuda.synchronize()
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(device.index) as clk:
+    with ClockSampler(device.index) as clk, torch.cuda.stream(stream):
         start.record(stream)
         graph.replay()
         end.record(stream)

@@ -98,20 +98,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// A row-major byte matrix (rows x row_bytes) read in boxes of box_rows x
-// box_bytes.
-convrot_status_t make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t row_bytes, int box_rows,
-                          int box_bytes, bool swizzle128) {
+// A row-major matrix (rows x cols elements of `dtype`, `elem_bytes` each) read
+// or written in boxes of box_rows x box_cols elements.
+convrot_status_t make_map(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, int64_t rows,
+                          int64_t cols, int box_rows, int box_cols, CUtensorMapSwizzle swizzle) {
     EncodeTiledFn fn = encode_fn();
     CR_REQUIRE(fn != nullptr, CONVROT_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows)};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * elem_bytes)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     CR_REQUIRE(r == CUDA_SUCCESS, CONVROT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
     return ok();
 }
@@ -207,16 +205,18 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *A, const
             done[dev] = true;
         }
     }
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, ty;
     const int64_t row_bytes = Cfg::W4 ? K / 2 : K;
     const int box_bytes = Cfg::W4 ? Cfg::BK / 2 : Cfg::BK;
-    CR_TRY(make_map(&ta, A, M, row_bytes, Cfg::BM, box_bytes, !Cfg::W4));
-    CR_TRY(make_map(&tb, B, N, row_bytes, Cfg::BN, box_bytes, !Cfg::W4));
+    const CUtensorMapSwizzle sw_in = Cfg::W4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+    CR_TRY(make_map(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, row_bytes, Cfg::BM, box_bytes, sw_in));
+    CR_TRY(make_map(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, row_bytes, Cfg::BN, box_bytes, sw_in));
+    CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, Cfg::CHUNK, CU_TENSOR_MAP_SWIZZLE_64B));
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
     const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
     convrot::gemm_i8_tcgen05_kernel<Cfg><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, st>>>(
-        ta, tb, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sx, sw,
-        static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out);
+        ta, tb, ty, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sx, sw,
+        static_cast<const __half *>(bias), acc_out);
     return launch_status("gemm_i8_tcgen05");
 }
 

@@ -14,8 +14,9 @@
 // 128 x BN, K step 128 bytes.
 //   warp 0      TMA producer (one elected lane): A and B tiles -> smem ring
 //   warp 1      TMEM allocator + MMA issuer (one lane): 4 x tcgen05.mma per K step
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, fp16, store
-//   warps 6-9   (W4A4 only) nibble -> byte converters between a packed ring
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator, scale, fp16, staged
+//               in shared memory and written by TMA bulk stores
+//   warps 10-13 (W4A4 only) nibble -> byte converters between a packed ring
 //               and the MMA ring
 // Two TMEM accumulators (2 x BN columns) let the epilogue of one tile overlap
 // the main loop of the next.  No TMA multicast is used anywhere.
@@ -35,19 +36,25 @@ struct GemmCfg {
     static constexpr int B_BYTES = BN * BK;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     // MMA ring depth and (W4A4) packed ring depth
-    static constexpr int STAGES = W4 ? (BN == 256 ? 3 : 4) : (BN == 256 ? 4 : 6);
+    static constexpr int STAGES = W4 ? (BN == 256 ? 2 : 3) : (BN == 256 ? 4 : 6);
     static constexpr int PSTAGES = W4 ? (BN == 256 ? 3 : 4) : 0;
     static constexpr int PA_BYTES = A_BYTES / 2;
     static constexpr int PB_BYTES = B_BYTES / 2;
     static constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
     static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int NUM_THREADS = W4 ? 320 : 192;
+    static constexpr int EPI_WARPS = 8;           // two per TMEM lane quarter, each half of the columns
+    static constexpr int EPI_COLS = BN / 2;       // columns per epilogue warp
+    static constexpr int CHUNK = 32;              // columns per TMEM load / output box
+    static constexpr int OUT_BOX_BYTES = 32 * CHUNK * 2;  // 32 rows x 32 fp16
+    static constexpr int OUT_BYTES = EPI_WARPS * 2 * OUT_BOX_BYTES;  // double-buffered per warp
+    static constexpr int FIRST_CONV_WARP = 2 + EPI_WARPS;
+    static constexpr int NUM_THREADS = 32 * (FIRST_CONV_WARP + (W4 ? 4 : 0));
     static constexpr int NUM_BARRIERS = 2 * STAGES + 2 * PSTAGES + 4 + 1;
-    static constexpr int SMEM_BYTES =
-        1024 /* alignment slack */ + STAGES * STAGE_BYTES + PSTAGES * PSTAGE_BYTES + NUM_BARRIERS * 8 + 16;
+    static constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * STAGE_BYTES + PSTAGES * PSTAGE_BYTES +
+                                      OUT_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t IDESC = idesc_i8(BM, BN);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
+    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
 };
 
 // Bounded wait used while draining: ignores the abort flag, still time-limited.
@@ -66,17 +73,54 @@ __device__ __forceinline__ uint4 widen_int4x16(uint2 p) {
                       __byte_perm(lo1, hi1, 0x7362));
 }
 
+// Dequantizes 8 accumulators of one row: fp16(fma(fp32(float(acc) * sx), sw[c], bias[c]))
+// (the final multiply-add is one explicit fused operation, so it rounds once).
+template <bool W4>
+__device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const float *__restrict__ sw,
+                                          const __half *__restrict__ bias, int col, int32_t *acc_vals) {
+    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(sw + col));
+    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(sw + col + 4));
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    float bv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (bias != nullptr) {
+        const uint4 braw = __ldg(reinterpret_cast<const uint4 *>(bias + col));
+        const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&bw[i]));
+            bv[2 * i] = p.x;
+            bv[2 * i + 1] = p.y;
+        }
+    }
+    uint32_t out[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int32_t a0 = W4 ? (static_cast<int32_t>(r[2 * i]) >> 8) : static_cast<int32_t>(r[2 * i]);
+        const int32_t a1 = W4 ? (static_cast<int32_t>(r[2 * i + 1]) >> 8) : static_cast<int32_t>(r[2 * i + 1]);
+        acc_vals[2 * i] = a0;
+        acc_vals[2 * i + 1] = a1;
+        float2 t = make_float2(__int2float_rn(a0), __int2float_rn(a1));
+        t = __fmul2_rn(t, make_float2(sxm, sxm));
+        t = __ffma2_rn(t, make_float2(wv[2 * i], wv[2 * i + 1]), make_float2(bv[2 * i], bv[2 * i + 1]));
+        const __half2 h = __floats2half2_rn(t.x, t.y);
+        out[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
-    gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                           int N, int K, const float *__restrict__ sx, const float *__restrict__ sw,
-                           const __half *__restrict__ bias, __half *__restrict__ Y, int32_t *__restrict__ acc_out) {
+    gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmY, int M, int N, int K, const float *__restrict__ sx,
+                           const float *__restrict__ sw, const __half *__restrict__ bias,
+                           int32_t *__restrict__ acc_out) {
     constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, PSTAGES = Cfg::PSTAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ring = smem;                                          // STAGES x (A | B), int8, 128B-swizzled
     uint8_t *pring = ring + STAGES * Cfg::STAGE_BYTES;             // PSTAGES x (A4 | B4), packed, dense rows
-    uint64_t *bars = reinterpret_cast<uint64_t *>(pring + PSTAGES * Cfg::PSTAGE_BYTES);
+    uint8_t *outbuf = pring + PSTAGES * Cfg::PSTAGE_BYTES;         // per epilogue warp: 2 x (32 x 32 fp16)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + Cfg::OUT_BYTES);
     uint64_t *full = bars;                                         // MMA ring: operands ready
     uint64_t *empty = full + STAGES;                               // MMA ring: slot consumed
     uint64_t *pfull = empty + STAGES;                              // packed ring: TMA landed
@@ -103,7 +147,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tmem_full[i], 1);
-            mbar_init(&tmem_empty[i], 128);
+            mbar_init(&tmem_empty[i], 32 * Cfg::EPI_WARPS);
         }
         mbar_init(drain, 1);
         *abort = 0;
@@ -112,6 +156,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -201,9 +246,14 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             umma_commit(drain);
             mbar_wait_drain(drain, 0);
         }
-    } else if (warp < 6) {
+    } else if (warp < Cfg::FIRST_CONV_WARP) {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        // Warp w reads TMEM lanes 32*(w%4) .. +31 (its hardware lane quarter)
+        // and columns [half * BN/2, (half+1) * BN/2) of the accumulator.
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        uint8_t *obuf = outbuf + (warp - 2) * 2 * Cfg::OUT_BOX_BYTES;
+        int ob = 0;
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const int acc = local & 1;
@@ -211,67 +261,56 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             if (!mbar_wait(&tmem_full[acc], acc_ph, abort)) break;
             tc_fence_after_sync();
             const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
-            const int row = tm * BM + q * 32 + lane;
+            const int row0 = tm * BM + q * 32;
+            const int row = row0 + lane;
             const bool row_ok = row < M;
             const float sxm = row_ok ? sx[row] : 0.0f;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                __syncwarp();  // tcgen05.ld is warp-collective
+            for (int c = 0; c < Cfg::EPI_COLS / Cfg::CHUNK; ++c) {
+                const int col_local = half * Cfg::EPI_COLS + c * Cfg::CHUNK;
                 uint32_t r[32];
-                tmem_ld_32x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, r);
+                __syncwarp();  // tcgen05.ld is warp-collective
+                tmem_ld_32x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + col_local, r);
                 tmem_ld_wait();
-                const int col0 = tn * BN + c * 32;
-                if (!row_ok || col0 >= N) continue;
+                if (c == Cfg::EPI_COLS / Cfg::CHUNK - 1) {
+                    // every TMEM read of this tile by this thread is complete
+                    tc_fence_before_sync();
+                    mbar_arrive(&tmem_empty[acc]);
+                }
+                const int col0 = tn * BN + col_local;
+                if (row0 >= M || col0 >= N) continue;  // whole box outside Y (warp-uniform)
+                // the store issued from this buffer two chunks ago must have read it
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+                uint8_t *box = obuf + ob * Cfg::OUT_BOX_BYTES;
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {  // 8 columns per 16-byte store
-                    const int col = col0 + 8 * g;
-                    if (col >= N) break;
-                    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(sw + col));
-                    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(sw + col + 4));
-                    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                    float bv[8];
-                    if (bias != nullptr) {
-                        const uint4 braw = __ldg(reinterpret_cast<const uint4 *>(bias + col));
-                        const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&bw[i]));
-                            bv[2 * i] = p.x;
-                            bv[2 * i + 1] = p.y;
+                for (int g = 0; g < 4; ++g) {
+                    int32_t av[8];
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (row_ok && col0 + 8 * g < N) {
+                        v = dequant8<Cfg::W4>(r + 8 * g, sxm, sw, bias, col0 + 8 * g, av);
+                        if (acc_out != nullptr) {
+                            int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0 + 8 * g);
+                            dst[0] = make_int4(av[0], av[1], av[2], av[3]);
+                            dst[1] = make_int4(av[4], av[5], av[6], av[7]);
                         }
                     }
-                    int32_t av[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int32_t raw = static_cast<int32_t>(r[8 * g + i]);
-                        av[i] = Cfg::W4 ? (raw >> 8) : raw;  // W4A4 operands carry 16 * code each
-                    }
-                    uint32_t out[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        float2 t = make_float2(__int2float_rn(av[2 * i]), __int2float_rn(av[2 * i + 1]));
-                        t = __fmul2_rn(t, make_float2(sxm, sxm));
-                        t = __fmul2_rn(t, make_float2(wv[2 * i], wv[2 * i + 1]));
-                        if (bias != nullptr) t = __fadd2_rn(t, make_float2(bv[2 * i], bv[2 * i + 1]));
-                        const __half2 h = __floats2half2_rn(t.x, t.y);
-                        out[i] = *reinterpret_cast<const uint32_t *>(&h);
-                    }
-                    *reinterpret_cast<uint4 *>(Y + static_cast<int64_t>(row) * N + col) =
-                        make_uint4(out[0], out[1], out[2], out[3]);
-                    if (acc_out != nullptr) {
-                        int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col);
-                        dst[0] = make_int4(av[0], av[1], av[2], av[3]);
-                        dst[1] = make_int4(av[4], av[5], av[6], av[7]);
-                    }
+                    // 64-byte rows, 16-byte chunk g stored at g ^ ((row >> 1) & 3) (64B swizzle)
+                    *reinterpret_cast<uint4 *>(box + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) = v;
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmY, box, col0, row0);
+                    bulk_commit_group();
+                }
+                ob ^= 1;
             }
-            __syncwarp();
-            tc_fence_before_sync();
-            mbar_arrive(&tmem_empty[acc]);
         }
+        if (lane == 0) bulk_wait_group_all();
     } else if (Cfg::W4) {
         // ------------------------------------------------------------ int4 -> int8 converters
-        const int ct = threadIdx.x - 192;  // 0..127
+        const int ct = threadIdx.x - 32 * Cfg::FIRST_CONV_WARP;  // 0..127
         int ps = 0, us = 0;
         uint32_t pph = 0, uph = 0;
         bool ok = true;

@@ -148,7 +148,8 @@ __device__ __forceinline__ float chunk_val(const float2 (&v)[2][8], int j, int e
     return j < 2 ? v[j][e].x : v[j - 2][e].y;
 }
 
-// Low byte of the bit pattern of (t + 1.5*2^23): rne(t) in 8-bit two's complement.
+// Low byte of the bit pattern of (t + 1.5*2^23) for an integer-rounded t:
+// rne(t) in 8-bit two's complement.
 __device__ __forceinline__ uint32_t code_bits(const float2 (&r)[2][8], int j, int e) {
     return __float_as_uint(chunk_val(r, j, e));
 }
@@ -185,6 +186,14 @@ __device__ __forceinline__ void store_codes(void *out_row, int elem0, const floa
                 pack_int4_chunk(r, j);
         }
     }
+}
+
+// clamp(rne(x * inv), qmin, qmax) as an exact integer-valued float: the fused
+// multiply-add rounds the exact product once onto the integer grid of
+// [2^23, 2^24), and removing the offset again is exact.
+__device__ __forceinline__ float quant_clamped(float x, float inv, int qmin, int qmax) {
+    const float r = __fsub_rn(__fmaf_rn(x, inv, kRoundMagic), kRoundMagic);
+    return fminf(fmaxf(r, static_cast<float>(qmin)), static_cast<float>(qmax));
 }
 
 // Largest power of two dividing L, at most 32: the lanes of one row that a
@@ -254,7 +263,7 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[h][e] = __fadd2_rn(__fmul2_rn(v[h][e], inv), f2(kRoundMagic));
+        for (int e = 0; e < 8; ++e) v[h][e] = __ffma2_rn(v[h][e], inv, f2(kRoundMagic));  // rne(x~ * inv), one rounding
     void *out_row = BITS == 8 ? static_cast<void *>(static_cast<int8_t *>(Xq) + row * K)
                               : static_cast<void *>(static_cast<uint8_t *>(Xq) + row * (K / 2));
     store_codes<BITS>(out_row, elem0, v);
@@ -343,8 +352,7 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
                     const float xs[2] = {v[h][e].x, v[h][e].y};
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
-                        const float t = __fmul_rn(xs[c], inv);
-                        const float q = fminf(fmaxf(rintf(t), static_cast<float>(qmin)), static_cast<float>(qmax));
+                        const float q = quant_clamped(xs[c], inv, qmin, qmax);
                         const double d = fma(-sd, static_cast<double>(q), static_cast<double>(xs[c]));
                         err = fma(d, d, err);
                     }
@@ -373,8 +381,8 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
     for (int h = 0; h < 2; ++h) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            float a = fminf(fmaxf(rintf(__fmul_rn(v[h][e].x, inv)), static_cast<float>(qmin)), static_cast<float>(qmax));
-            float b = fminf(fmaxf(rintf(__fmul_rn(v[h][e].y, inv)), static_cast<float>(qmin)), static_cast<float>(qmax));
+            const float a = quant_clamped(v[h][e].x, inv, qmin, qmax);
+            const float b = quant_clamped(v[h][e].y, inv, qmin, qmax);
             // re-encode the (exact, small) integers with the rounding magic so
             // that the packers can take their low bytes
             q[h][e] = make_float2(__fadd_rn(a, kRoundMagic), __fadd_rn(b, kRoundMagic));
