@@ -149,6 +149,27 @@ convrot_status_t convrot_gemm_w4a4(const uint8_t *Xq, const float *x_scale, int6
                                    int32_t *acc_out, void *stream);
 
 /*
+ * W8A8 ConvRot linear that allocates nothing and takes no workspace.  The
+ * source pages have no counterpart: this exists for callers that cannot
+ * allocate device memory (a plugin whose host framework owns the GPU's memory
+ * and offers no allocator, or a path where an allocation is not allowed).
+ * Arguments and results are those of convrot_linear_w8a8 without
+ * workspace / workspace_bytes.
+ *   - Scratch (activation codes and scales) lives in one 16 MiB array built
+ *     into the library; every GPU that loads the library holds it until the
+ *     process exits.  Calls needing more (M*K + 4*M bytes, each rounded up to
+ *     256) return CONVROT_ERR_WORKSPACE without launching.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls on a device share the array and leave the last call's codes in
+ *     it; nothing needs to start at zero.  Calls whose kernels overlap on the
+ *     GPU (different streams, no ordering between them) race on it.
+ */
+convrot_status_t convrot_linear_w8a8_noalloc(const void *X, int64_t M, int64_t K, const int8_t *Wq,
+                                             const float *w_scale, int64_t N, const void *bias, int block,
+                                             void *Y, void *stream);
+
+/*
  * Synchronizes `stream`, then returns and clears the sticky device-side
  * status of the current device: CONVROT_OK, CONVROT_ERR_TIMEOUT if a kernel
  * abandoned a wait since the last query, or CONVROT_ERR_CUDA if the stream

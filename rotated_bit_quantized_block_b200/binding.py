@@ -23,6 +23,7 @@ EXPORTED = (
     "convrot_quantize_weight", "convrot_rotate_quant_act", "convrot_workspace_bytes",
     "convrot_linear_w8a8", "convrot_linear_w4a4", "convrot_gemm_w8a8", "convrot_gemm_w4a4",
     "convrot_device_status", "convrot_status_string", "convrot_last_error", "convrot_version",
+    "convrot_linear_w8a8_noalloc",
 )
 
 
@@ -54,6 +55,7 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
             "convrot_linear_w4a4": (i32, [P, i64, i64, P, P, i64, P, i32, P, P, sz, P]),
             "convrot_gemm_w8a8": (i32, [P, P, i64, P, P, i64, i64, P, P, P, P]),
             "convrot_gemm_w4a4": (i32, [P, P, i64, P, P, i64, i64, P, P, P, P]),
+            "convrot_linear_w8a8_noalloc": (i32, [P, i64, i64, P, P, i64, P, i32, P, P]),
             "convrot_device_status": (i32, [P]),
             "convrot_status_string": (ctypes.c_char_p, [i32]),
             "convrot_last_error": (ctypes.c_char_p, []),
@@ -184,6 +186,21 @@ def convrot_gemm_w8a8(Xq, x_scale, Wq, w_scale, bias=None, Y=None, acc_out=None,
 def convrot_gemm_w4a4(Xq, x_scale, Wq, w_scale, bias=None, Y=None, acc_out=None, stream=None):
     """Integer GEMM + dequant epilogue on packed int4 codes (Xq M x K/2, Wq N x K/2)."""
     return _gemm("convrot_gemm_w4a4", Xq, x_scale, Wq, w_scale, Xq.shape[1] * 2, bias, Y, acc_out, stream)
+
+
+def convrot_linear_w8a8_noalloc(X, Wq, w_scale, block, bias=None, Y=None, stream=None):
+    """W8A8 ConvRot linear without a workspace: for callers that may not allocate
+    device memory.  The codes and scales go to a fixed 16 MiB array inside the
+    library (shared by all calls on a device), so M*K is limited to about 16 MiB."""
+    _dev(X, "X")
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    st = load_library().convrot_linear_w8a8_noalloc(_ptr(X), M, K, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), block,
+                                                    _ptr(Y), _stream(stream))
+    _check(st)
+    return Y
 
 
 def convrot_device_status(stream=None):

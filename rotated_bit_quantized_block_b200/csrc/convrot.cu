@@ -391,6 +391,54 @@ convrot_status_t convrot_gemm_w4a4(const uint8_t *Xq, const float *x_scale, int6
     return gemm_impl(true, Xq, x_scale, M, Wq, w_scale, N, K, bias, Y, acc_out, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free W8A8 linear.  Some callers cannot allocate device memory at
+// all -- a plugin inside a host framework that owns every byte of the GPU and
+// hands out no allocator, or a latency-critical path where an allocation (and
+// the device synchronization it can imply) is not allowed.  For them this entry
+// point keeps the activation codes and per-token scales in one fixed array
+// compiled into the library instead of a caller workspace.
+// ---------------------------------------------------------------------------
+
+static constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB on every device that loads the library
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+static void *g_noalloc_ptr[kMaxDevices];
+static std::mutex g_noalloc_mutex;
+
+convrot_status_t convrot_linear_w8a8_noalloc(const void *X, int64_t M, int64_t K, const int8_t *Wq,
+                                             const float *w_scale, int64_t N, const void *bias, int block, void *Y,
+                                             void *stream) {
+    g_last_error.clear();
+    CR_TRY(check_shape(M, K, block, "M"));
+    CR_REQUIRE(N >= 0 && N < (int64_t(1) << 31) && N % 8 == 0, CONVROT_ERR_INVALID_ARG,
+               "N = %lld must be a multiple of 8 in [0, 2^31)", static_cast<long long>(N));
+    if (M == 0 || N == 0) return ok();
+    const size_t need = convrot_workspace_bytes(M, K, 8);
+    CR_REQUIRE(need <= kNoAllocScratchBytes, CONVROT_ERR_WORKSPACE,
+               "M = %lld, K = %lld needs %zu bytes of scratch; the built-in array holds %zu "
+               "(use convrot_linear_w8a8 with a workspace)",
+               static_cast<long long>(M), static_cast<long long>(K), need, kNoAllocScratchBytes);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    CR_REQUIRE(dev >= 0 && dev < kMaxDevices, CONVROT_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    void *scratch = nullptr;
+    {
+        // The array's name is only a host-side stand-in: its device address is
+        // looked up once per device, with that device current.
+        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+        if (g_noalloc_ptr[dev] == nullptr) {
+            void *p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            CR_REQUIRE(e == cudaSuccess && p != nullptr, CONVROT_ERR_CUDA, "cudaGetSymbolAddress: %s",
+                       cudaGetErrorString(e));
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    return linear_impl(8, X, M, K, Wq, w_scale, N, bias, block, Y, scratch, kNoAllocScratchBytes, stream);
+}
+
 convrot_status_t convrot_device_status(void *stream) {
     g_last_error.clear();
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
