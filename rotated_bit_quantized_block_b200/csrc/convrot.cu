@@ -211,7 +211,7 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *A, const
     const CUtensorMapSwizzle sw_in = Cfg::W4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
     CR_TRY(make_map(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, row_bytes, Cfg::BM, box_bytes, sw_in));
     CR_TRY(make_map(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, row_bytes, Cfg::BN, box_bytes, sw_in));
-    CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, Cfg::CHUNK, CU_TENSOR_MAP_SWIZZLE_64B));
+    CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, Cfg::CHUNK, CU_TENSOR_MAP_SWIZZLE_128B));
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
     const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
     convrot::gemm_i8_tcgen05_kernel<Cfg><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, st>>>(

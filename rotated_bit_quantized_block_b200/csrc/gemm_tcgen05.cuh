@@ -44,14 +44,15 @@ struct GemmCfg {
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int EPI_WARPS = 8;           // two per TMEM lane quarter, each half of the columns
     static constexpr int EPI_COLS = BN / 2;       // columns per epilogue warp
-    static constexpr int CHUNK = 32;              // columns per TMEM load / output box
-    static constexpr int OUT_BOX_BYTES = 32 * CHUNK * 2;  // 32 rows x 32 fp16
-    static constexpr int OUT_BYTES = EPI_WARPS * 2 * OUT_BOX_BYTES;  // double-buffered per warp
+    static constexpr int CHUNK = 64;              // columns per output box (two 32-column TMEM loads)
+    static constexpr int OUT_BOX_BYTES = 32 * CHUNK * 2;  // 32 rows x 64 fp16, 128-byte rows
+    static constexpr int OUT_BYTES = EPI_WARPS * OUT_BOX_BYTES;  // one box per epilogue warp
+    static constexpr int SCALE_BYTES = BN * 4 + BN * 2;        // the tile's w_scale (fp32) and bias (fp16)
     static constexpr int FIRST_CONV_WARP = 2 + EPI_WARPS;
     static constexpr int NUM_THREADS = 32 * (FIRST_CONV_WARP + (W4 ? 4 : 0));
-    static constexpr int NUM_BARRIERS = 2 * STAGES + 2 * PSTAGES + 4 + 1;
+    static constexpr int NUM_BARRIERS = 2 * STAGES + 2 * PSTAGES + 4 + 1 + 2;
     static constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * STAGE_BYTES + PSTAGES * PSTAGE_BYTES +
-                                      OUT_BYTES + NUM_BARRIERS * 8 + 16;
+                                      OUT_BYTES + SCALE_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t IDESC = idesc_i8(BM, BN);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
@@ -75,23 +76,15 @@ __device__ __forceinline__ uint4 widen_int4x16(uint2 p) {
 
 // Dequantizes 8 accumulators of one row: fp16(fma(fp32(float(acc) * sx), sw[c], bias[c]))
 // (the final multiply-add is one explicit fused operation, so it rounds once).
+// sw_s / bias_s point at the tile's scales staged in shared memory.
 template <bool W4>
-__device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const float *__restrict__ sw,
-                                          const __half *__restrict__ bias, int col, int32_t *acc_vals) {
-    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(sw + col));
-    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(sw + col + 4));
+__device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const float *sw_s, const __half *bias_s,
+                                          int32_t *acc_vals) {
+    const float4 w0 = *reinterpret_cast<const float4 *>(sw_s);
+    const float4 w1 = *reinterpret_cast<const float4 *>(sw_s + 4);
     const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    float bv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (bias != nullptr) {
-        const uint4 braw = __ldg(reinterpret_cast<const uint4 *>(bias + col));
-        const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&bw[i]));
-            bv[2 * i] = p.x;
-            bv[2 * i + 1] = p.y;
-        }
-    }
+    const uint4 braw = *reinterpret_cast<const uint4 *>(bias_s);
+    const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
     uint32_t out[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -99,9 +92,10 @@ __device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const fl
         const int32_t a1 = W4 ? (static_cast<int32_t>(r[2 * i + 1]) >> 8) : static_cast<int32_t>(r[2 * i + 1]);
         acc_vals[2 * i] = a0;
         acc_vals[2 * i + 1] = a1;
+        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&bw[i]));
         float2 t = make_float2(__int2float_rn(a0), __int2float_rn(a1));
         t = __fmul2_rn(t, make_float2(sxm, sxm));
-        t = __ffma2_rn(t, make_float2(wv[2 * i], wv[2 * i + 1]), make_float2(bv[2 * i], bv[2 * i + 1]));
+        t = __ffma2_rn(t, make_float2(wv[2 * i], wv[2 * i + 1]), b);
         const __half2 h = __floats2half2_rn(t.x, t.y);
         out[i] = *reinterpret_cast<const uint32_t *>(&h);
     }
@@ -119,8 +113,10 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ring = smem;                                          // STAGES x (A | B), int8, 128B-swizzled
     uint8_t *pring = ring + STAGES * Cfg::STAGE_BYTES;             // PSTAGES x (A4 | B4), packed, dense rows
-    uint8_t *outbuf = pring + PSTAGES * Cfg::PSTAGE_BYTES;         // per epilogue warp: 2 x (32 x 32 fp16)
-    uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + Cfg::OUT_BYTES);
+    uint8_t *outbuf = pring + PSTAGES * Cfg::PSTAGE_BYTES;         // per epilogue warp: 32 x 64 fp16 box
+    float *sw_s = reinterpret_cast<float *>(outbuf + Cfg::OUT_BYTES);          // [BN] tile w_scale
+    __half *bias_s = reinterpret_cast<__half *>(sw_s + BN);                     // [BN] tile bias
+    uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + Cfg::OUT_BYTES + Cfg::SCALE_BYTES);
     uint64_t *full = bars;                                         // MMA ring: operands ready
     uint64_t *empty = full + STAGES;                               // MMA ring: slot consumed
     uint64_t *pfull = empty + STAGES;                              // packed ring: TMA landed
@@ -128,7 +124,9 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     uint64_t *tmem_full = pempty + PSTAGES;                        // [2] accumulator ready
     uint64_t *tmem_empty = tmem_full + 2;                          // [2] accumulator drained
     uint64_t *drain = tmem_empty + 2;                              // MMA completion at exit
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *scale_ready = drain + 1;                             // tile scales staged in smem
+    uint64_t *scale_free = scale_ready + 1;                        // tile scales no longer read
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(scale_free + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -150,6 +148,8 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             mbar_init(&tmem_empty[i], 32 * Cfg::EPI_WARPS);
         }
         mbar_init(drain, 1);
+        mbar_init(scale_ready, 32 * Cfg::EPI_WARPS);
+        mbar_init(scale_free, 32 * Cfg::EPI_WARPS);
         *abort = 0;
         fence_mbarrier_init();
     }
@@ -249,17 +249,43 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     } else if (warp < Cfg::FIRST_CONV_WARP) {
         // ------------------------------------------------------------ epilogue
         // Warp w reads TMEM lanes 32*(w%4) .. +31 (its hardware lane quarter)
-        // and columns [half * BN/2, (half+1) * BN/2) of the accumulator.
+        // and columns [half * BN/2, (half+1) * BN/2) of the accumulator.  The
+        // tile's w_scale / bias are prefetched into registers one tile ahead
+        // (one column per thread) and staged in shared memory at tile start.
+        const int ew = warp - 2;  // 0..7
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;
-        uint8_t *obuf = outbuf + (warp - 2) * 2 * Cfg::OUT_BOX_BYTES;
-        int ob = 0;
+        const int half = ew >> 2;
+        uint8_t *box = outbuf + ew * Cfg::OUT_BOX_BYTES;
+        const int scol = ew * 32 + lane;  // the tile column this thread stages (valid if < BN)
+        auto load_scales = [&](int t, float &wv, __half &bv) {
+            wv = 0.0f;
+            bv = __float2half_rn(0.0f);
+            if (t < num_tiles && scol < BN) {
+                const int col = (t - (t / tiles_n) * tiles_n) * BN + scol;
+                if (col < N) {
+                    wv = __ldg(sw + col);
+                    if (bias != nullptr) bv = bias[col];
+                }
+            }
+        };
+        float next_w;
+        __half next_b;
+        load_scales(blockIdx.x, next_w, next_b);
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const int acc = local & 1;
             const uint32_t acc_ph = (local >> 1) & 1;
             if (!mbar_wait(&tmem_full[acc], acc_ph, abort)) break;
             tc_fence_after_sync();
+            // every epilogue thread is done with the previous tile's scales
+            if (local > 0 && !mbar_wait(scale_free, (local - 1) & 1, abort)) break;
+            if (scol < BN) {
+                sw_s[scol] = next_w;
+                bias_s[scol] = next_b;
+            }
+            mbar_arrive(scale_ready);
+            if (!mbar_wait(scale_ready, local & 1, abort)) break;
+            load_scales(tile + gridDim.x, next_w, next_b);
             const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
             const int row0 = tm * BM + q * 32;
             const int row = row0 + lane;
@@ -268,9 +294,11 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
 #pragma unroll 1
             for (int c = 0; c < Cfg::EPI_COLS / Cfg::CHUNK; ++c) {
                 const int col_local = half * Cfg::EPI_COLS + c * Cfg::CHUNK;
-                uint32_t r[32];
+                uint32_t r[2][32];
                 __syncwarp();  // tcgen05.ld is warp-collective
-                tmem_ld_32x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + col_local, r);
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + col_local;
+                tmem_ld_32x32(taddr, r[0]);
+                tmem_ld_32x32(taddr + 32, r[1]);
                 tmem_ld_wait();
                 if (c == Cfg::EPI_COLS / Cfg::CHUNK - 1) {
                     // every TMEM read of this tile by this thread is complete
@@ -279,24 +307,24 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                 }
                 const int col0 = tn * BN + col_local;
                 if (row0 >= M || col0 >= N) continue;  // whole box outside Y (warp-uniform)
-                // the store issued from this buffer two chunks ago must have read it
-                if (lane == 0) bulk_wait_group_read<1>();
+                // the store issued from this box last time must have read it
+                if (lane == 0) bulk_wait_group_read<0>();
                 __syncwarp();
-                uint8_t *box = obuf + ob * Cfg::OUT_BOX_BYTES;
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
+                for (int g = 0; g < 8; ++g) {  // 8 columns per 16-byte chunk
                     int32_t av[8];
                     uint4 v = make_uint4(0, 0, 0, 0);
                     if (row_ok && col0 + 8 * g < N) {
-                        v = dequant8<Cfg::W4>(r + 8 * g, sxm, sw, bias, col0 + 8 * g, av);
+                        v = dequant8<Cfg::W4>(r[g >> 2] + 8 * (g & 3), sxm, sw_s + col_local + 8 * g,
+                                              bias_s + col_local + 8 * g, av);
                         if (acc_out != nullptr) {
                             int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0 + 8 * g);
                             dst[0] = make_int4(av[0], av[1], av[2], av[3]);
                             dst[1] = make_int4(av[4], av[5], av[6], av[7]);
                         }
                     }
-                    // 64-byte rows, 16-byte chunk g stored at g ^ ((row >> 1) & 3) (64B swizzle)
-                    *reinterpret_cast<uint4 *>(box + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) = v;
+                    // 128-byte rows, 16-byte chunk g stored at g ^ (row & 7) (128B swizzle)
+                    *reinterpret_cast<uint4 *>(box + lane * 128 + ((g ^ (lane & 7)) << 4)) = v;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -304,8 +332,8 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     tma_store_2d(&tmY, box, col0, row0);
                     bulk_commit_group();
                 }
-                ob ^= 1;
             }
+            mbar_arrive(scale_free);
         }
         if (lane == 0) bulk_wait_group_all();
     } else if (Cfg::W4) {
