@@ -127,11 +127,14 @@ class Replica:
         return sum(it["X"].nbytes + it["Y"].nbytes + it["Wq"].nbytes + it["ws"].nbytes for it in self.items)
 
 
-def run_step(w, rep, stream, gemm_events=None):
+def run_step(w, rep, stream, events=None):
     """One pass over every linear: rotate+quant kernel, then GEMM+dequant kernel.
 
     The two kernels are launched through their own entry points (the same
-    launches convrot_linear_* makes) so that the GEMM can be bracketed by events.
+    launches convrot_linear_* makes).  With ``events`` (per linear: act start,
+    act end = GEMM start, GEMM end) every kernel is bracketed for per-kernel
+    timing; event nodes between kernels also stop the next kernel from starting
+    early, so the throughput pass runs without them.
     """
     for i, it in enumerate(rep.items):
         lin = it["lin"]
@@ -140,13 +143,15 @@ def run_step(w, rep, stream, gemm_events=None):
         off = (code_bytes + 255) // 256 * 256
         xq = ws[:code_bytes].view(torch.int8 if w.bits == 8 else torch.uint8).view(w.M, -1)
         xs = ws[off:off + 4 * w.M].view(torch.float32)
+        if events is not None:
+            events[i][0].record(stream)
         cr.convrot_rotate_quant_act(it["X"], w.block, w.bits, Xq=xq, x_scale=xs, stream=stream)
-        if gemm_events is not None:
-            gemm_events[i][0].record(stream)
+        if events is not None:
+            events[i][1].record(stream)
         gemm = cr.convrot_gemm_w8a8 if w.bits == 8 else cr.convrot_gemm_w4a4
         gemm(xq, xs, it["Wq"], it["sw"], Y=it["Y"], stream=stream)
-        if gemm_events is not None:
-            gemm_events[i][1].record(stream)
+        if events is not None:
+            events[i][2].record(stream)
 
 
 def run_step_linear(w, rep, stream):
@@ -270,17 +275,23 @@ def ours_arm(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     cr.convrot_device_status(stream)
 
-    # capture the K timed steps as one graph, with an event pair around every GEMM
+    # capture the K timed steps twice: as they run (throughput), and with events
+    # around every kernel (per-kernel durations for the rooflines)
     n_lin = len(w.linears)
-    events = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(n_lin)]
+    events = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(n_lin)]
               for _ in range(args.steps)]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for s in range(args.steps):
-            run_step(w, reps[s % 2], stream, gemm_events=events[s])
+            run_step(w, reps[s % 2], stream)
+    graph_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ev, stream=stream):
+        for s in range(args.steps):
+            run_step(w, reps[s % 2], stream, events=events[s])
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
-        graph.replay()  # one untimed replay of the captured steps
+        graph.replay()  # untimed replays of the captured steps
+        graph_ev.replay()
     torch.cuda.synchronize()
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -292,10 +303,13 @@ def ours_arm(args, w, rank, world, local_rank):
         graph.replay()
         end.record(stream)
         torch.cuda.synchronize()
+        graph_ev.replay()
+        torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     elapsed_ms = start.elapsed_time(end)
-    gemm_ms = [[events[s][i][0].elapsed_time(events[s][i][1]) for i in range(n_lin)] for s in range(args.steps)]
+    act_ms = [[events[s][i][0].elapsed_time(events[s][i][1]) for i in range(n_lin)] for s in range(args.steps)]
+    gemm_ms = [[events[s][i][1].elapsed_time(events[s][i][2]) for i in range(n_lin)] for s in range(args.steps)]
     cr.convrot_device_status(stream)
     clocks = clk.summary()
 
@@ -340,18 +354,27 @@ def ours_arm(args, w, rank, world, local_rank):
     achieved_tops = gemm_ops_total / (gemm_total_ms / 1000.0) / 1e12
     int8_peak = 2.0 * peaks["bf16_tflops"]  # dense int8 = 2 x dense bf16 (4.5 vs 2.25 POPS nominal)
     per_linear_ms = [statistics.mean(gemm_ms[s][i] for s in range(args.steps)) for i in range(n_lin)]
-    act_ms_step = ms_per_step - sum(per_linear_ms)
-    act_bytes_step = sum(w.M * l.K * 2 + w.M * l.K * w.bits // 8 + 4 * w.M for l in w.linears)
+    per_linear_act_ms = [statistics.mean(act_ms[s][i] for s in range(args.steps)) for i in range(n_lin)]
     roofline = {
         "bound": "tensor", "achieved": achieved_tops, "peak": int8_peak, "unit": "TOPS",
         "frac": achieved_tops / int8_peak, "traffic": None,
         "kernel": "gemm_i8_tcgen05 (int8 x int8 -> int32, fused dequant epilogue)",
         "peak_note": f"dense int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s",
+        "timing": "second timed pass of the same steps with CUDA events around every kernel launch",
         "per_linear_ms": {l.name: round(t, 5) for l, t in zip(w.linears, per_linear_ms)},
         "per_linear_tops": {l.name: round(2 * w.M * l.K * l.N / (t / 1000) / 1e12, 1)
                             for l, t in zip(w.linears, per_linear_ms)},
     }
-    act_gbs = act_bytes_step / (act_ms_step / 1000.0) / 1e9 if act_ms_step > 0 else None
+    act_bytes = [w.M * l.K * 2 + w.M * l.K * w.bits // 8 + 4 * w.M for l in w.linears]
+    act_total_ms = sum(per_linear_act_ms)
+    act_gbs = sum(act_bytes) / (act_total_ms / 1000.0) / 1e9
+    rotate_quant = {
+        "bound": "hbm", "achieved": act_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": act_gbs / peaks["hbm_gbs"], "kernel": "act_rotate_quant",
+        "per_linear_ms": {l.name: round(t, 5) for l, t in zip(w.linears, per_linear_act_ms)},
+        "per_linear_gbs": {l.name: round(b / (t / 1000) / 1e9, 1)
+                           for l, b, t in zip(w.linears, act_bytes, per_linear_act_ms)},
+    }
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -360,10 +383,7 @@ def ours_arm(args, w, rank, world, local_rank):
                                         f"{per_set / 2**20:.0f} MiB each (L2 {L2_BYTES >> 20} MiB)"),
         "tops": ops_step * world * args.steps / (elapsed_ms / 1000.0) / 1e12,
         "roofline": roofline,
-        "rotate_quant": {"bound": "hbm", "ms_per_step": act_ms_step, "achieved_gbs": act_gbs,
-                         "peak_gbs": peaks["hbm_gbs"],
-                         "frac": act_gbs / peaks["hbm_gbs"] if act_gbs else None,
-                         "note": "step time minus the GEMM launches (includes launch gaps)"},
+        "rotate_quant": rotate_quant,
         "offline_weight_quant_ms": weight_quant_ms,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "convrot_linear_* with pinned-host X copied in and Y copied out every step"},

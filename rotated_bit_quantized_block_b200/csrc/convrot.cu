@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/convrot.h"
 #include "device_utils.cuh"
@@ -137,7 +138,8 @@ convrot_status_t check_bits(int bits) {
         if (st_ != CONVROT_OK) return st_;    \
     } while (0)
 
-// Rows per CTA and threads per CTA of the rotation kernels.
+// Rows per CTA and threads per CTA of the rotation kernels (K/32 threads per
+// row, at least 256 threads per CTA where K allows).
 void rotate_geometry(int64_t K, int *rows, int *threads) {
     const int L = static_cast<int>(K / convrot::kElemsPerThread);
     int R = L >= 256 ? 1 : 256 / L;
@@ -146,27 +148,95 @@ void rotate_geometry(int64_t K, int *rows, int *threads) {
     *threads = ((R * L + 31) / 32) * 32;
 }
 
+// For the activation kernel: the rows per CTA that minimise (waves x rows per
+// CTA) given the kernel's real occupancy, so that a problem that fits in one
+// wave is launched as exactly one wave (a partial second wave would repeat the
+// whole load-compute-store latency).
+template <typename Kern>
+void act_geometry(Kern kernel, int sms, int64_t M, int64_t K, int *rows, int *threads) {
+    const int L = static_cast<int>(K / convrot::kElemsPerThread);
+    int R0, T0;
+    rotate_geometry(K, &R0, &T0);
+    int best_R = R0, best_T = T0;
+    int64_t best_cost = -1;
+    const int rmax_threads = 1024 / L;
+    const int r_hi = rmax_threads < convrot::kMaxRowsPerCta ? rmax_threads : convrot::kMaxRowsPerCta;
+    for (int R = R0; R <= r_hi; ++R) {
+        const int T = ((R * L + 31) / 32) * 32;
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, T, convrot::act_smem_bytes(T)) !=
+                cudaSuccess ||
+            per_sm <= 0) {
+            cudaGetLastError();
+            continue;
+        }
+        const int64_t ctas = (M + R - 1) / R;
+        const int64_t cap = static_cast<int64_t>(per_sm) * sms;
+        const int64_t waves = (ctas + cap - 1) / cap;
+        const int64_t cost = waves * R;
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best_R = R;
+            best_T = T;
+        }
+    }
+    *rows = best_R;
+    *threads = best_T;
+}
+
+// Launches with programmatic stream serialization: the kernel may begin while
+// the previous kernel in the stream finishes; it waits (griddepcontrol.wait)
+// before touching memory that kernel may use.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int LOG2B, int BITS>
-void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st) {
+void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms, int dev) {
+    auto kern = convrot::act_rotate_quant_kernel<LOG2B, BITS>;
+    {
+        static bool configured[kMaxDevices];
+        static std::mutex mu;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!configured[dev]) {
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, convrot::act_smem_bytes(1024));
+            // the largest shared-memory carve-out, so occupancy is limited by registers only
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            configured[dev] = true;
+        }
+    }
     int R, T;
-    rotate_geometry(K, &R, &T);
+    act_geometry(kern, sms, M, K, &R, &T);
     const int64_t grid = (M + R - 1) / R;
-    convrot::act_rotate_quant_kernel<LOG2B, BITS><<<static_cast<unsigned>(grid), T, 0, st>>>(
-        static_cast<const __half *>(X), M, static_cast<int>(K), R, Xq, xs);
+    launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(T), static_cast<size_t>(convrot::act_smem_bytes(T)), st,
+               static_cast<const __half *>(X), M, static_cast<int>(K), R, Xq, xs);
 }
 
 template <int BITS>
-void dispatch_act(int log2b, const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st) {
+void dispatch_act(int log2b, const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms,
+                  int dev) {
     switch (log2b) {
-        case 0: launch_act<0, BITS>(X, M, K, Xq, xs, st); break;
-        case 1: launch_act<1, BITS>(X, M, K, Xq, xs, st); break;
-        case 2: launch_act<2, BITS>(X, M, K, Xq, xs, st); break;
-        case 3: launch_act<3, BITS>(X, M, K, Xq, xs, st); break;
-        case 4: launch_act<4, BITS>(X, M, K, Xq, xs, st); break;
-        case 5: launch_act<5, BITS>(X, M, K, Xq, xs, st); break;
-        case 6: launch_act<6, BITS>(X, M, K, Xq, xs, st); break;
-        case 7: launch_act<7, BITS>(X, M, K, Xq, xs, st); break;
-        default: launch_act<8, BITS>(X, M, K, Xq, xs, st); break;
+        case 0: launch_act<0, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 1: launch_act<1, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 2: launch_act<2, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 3: launch_act<3, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 4: launch_act<4, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 5: launch_act<5, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 6: launch_act<6, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 7: launch_act<7, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
+        default: launch_act<8, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
     }
 }
 
@@ -181,10 +251,10 @@ void launch_weight(const void *W, int dtype, int64_t N, int64_t K, int bits, int
 }
 
 convrot_status_t rotate_quant_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, void *Xq,
-                                       float *x_scale, cudaStream_t st) {
+                                       float *x_scale, cudaStream_t st, int sms, int dev) {
     const int log2b = ilog2(block);
-    if (bits == 8) dispatch_act<8>(log2b, X, M, K, Xq, x_scale, st);
-    else dispatch_act<4>(log2b, X, M, K, Xq, x_scale, st);
+    if (bits == 8) dispatch_act<8>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
+    else dispatch_act<4>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
     return launch_status("act_rotate_quant");
 }
 
@@ -214,9 +284,9 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *A, const
     CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, Cfg::CHUNK, CU_TENSOR_MAP_SWIZZLE_128B));
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
     const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
-    convrot::gemm_i8_tcgen05_kernel<Cfg><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, st>>>(
-        ta, tb, ty, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sx, sw,
-        static_cast<const __half *>(bias), acc_out);
+    launch_pdl(convrot::gemm_i8_tcgen05_kernel<Cfg>, dim3(grid), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, ta, tb,
+               ty, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sx, sw,
+               static_cast<const __half *>(bias), acc_out);
     return launch_status("gemm_i8_tcgen05");
 }
 
@@ -322,7 +392,7 @@ convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, i
     int dev;
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
-    return rotate_quant_act_impl(X, M, K, block, bits, Xq, x_scale, static_cast<cudaStream_t>(stream));
+    return rotate_quant_act_impl(X, M, K, block, bits, Xq, x_scale, static_cast<cudaStream_t>(stream), info->sms, dev);
 }
 
 static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t K, const void *Wq,
@@ -347,7 +417,7 @@ static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t 
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    CR_TRY(rotate_quant_act_impl(X, M, K, block, bits, xq, xs, st));
+    CR_TRY(rotate_quant_act_impl(X, M, K, block, bits, xq, xs, st, info->sms, dev));
     if (bits == 8) return launch_gemm<false>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
     return launch_gemm<true>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
 }

@@ -207,6 +207,19 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 // Waits until every committed bulk group has completed.
 __device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel in the stream is still running.  pdl_wait() blocks until that
+// kernel has completed and its memory is visible; nothing produced or read by
+// it may be touched before.  pdl_launch_dependents() lets the next kernel start
+// its own prologue early (it still waits for this kernel's completion).
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {

@@ -166,6 +166,8 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // the codes and scales may come from the previous kernel
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer

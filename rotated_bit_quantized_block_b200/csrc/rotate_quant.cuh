@@ -205,16 +205,47 @@ __host__ __device__ __forceinline__ int reduce_width(int L) {
 
 // ---------------------------------------------------------------------------
 // Online activation path: X (fp16, M x K) -> codes + per-token scales.
-// One CTA handles `rows` consecutive rows with L = K/32 threads each; the
-// block is padded to a multiple of 32 threads (padding threads only join the
-// shuffles and barriers).
+//
+// One CTA handles `rows` consecutive rows with L = K/32 threads each (the
+// block is padded to a multiple of 32 threads; padding threads only join the
+// barriers).  Every thread issues its four 16-byte loads up front.  A thread
+// owns 32 elements of a 128-element group in two layouts:
+//   layout A: element 8p + 32j + e (chunks j = 0..3 of 8 e; p = thread in the
+//             group), packed as float2 (e, e+1): butterflies on bits 1, 2, 5, 6;
+//   layout B: element 32p + i (i = 0..31 contiguous), packed as float2
+//             (i, i+2): butterflies on bits 0, 3, 4 (bit 7, blocks of 256,
+//             between lanes l^4).
+// A -> B goes through a swizzled, bank-conflict-free 528-byte buffer per
+// group, so every butterfly runs on the packed fp32x2 pipe and each thread
+// ends with 32 contiguous codes (16-byte stores).  The 1/sqrt(b) factor is
+// folded into the per-row code factor (exact when b is a power of 4).
 // ---------------------------------------------------------------------------
+constexpr int kXposeGroupBytes = 33 * 16;  // 32 16-byte units + 1 unit of padding
+
+// 16-byte unit u (0..31) of a group's transpose buffer lives at this unit slot.
+__device__ __forceinline__ int xpose_slot(int u) { return (u & 24) | ((u & 7) ^ ((u >> 2) & 6)); }
+
+__device__ __forceinline__ void bfly2(float2 &a, float2 &b) {
+    const float2 s = __fadd2_rn(a, b);
+    b = sub2(a, b);
+    a = s;
+}
+
+// max(m, |x|, |y|)
+__device__ __forceinline__ float absmax3(float m, float x, float y) {
+    return fmaxf(m, fmaxf(fabsf(x), fabsf(y)));
+}
+
+// Dynamic shared memory of the activation kernel for a block of `threads`.
+__host__ __device__ constexpr int act_smem_bytes(int threads) { return (threads / 4) * kXposeGroupBytes; }
+
 template <int LOG2B, int BITS>
 __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__restrict__ X, int64_t M, int K,
                                                                 int rows, void *__restrict__ Xq,
                                                                 float *__restrict__ x_scale) {
+    extern __shared__ __align__(16) uint8_t act_smem[];
     __shared__ unsigned int s_amax[kMaxRowsPerCta];
-    __shared__ float s_inv[kMaxRowsPerCta];
+    __shared__ float s_fac[kMaxRowsPerCta];
     const int L = K / kElemsPerThread;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -222,51 +253,168 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
     const int l = tid - r * L;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * rows + r;
     const bool active = (r < rows) && (row < M);
-    const int elem0 = 128 * (l >> 2) + 8 * (l & 3);
+    const int g = l >> 2, p = l & 3;
     constexpr float qmax = BITS == 8 ? 127.0f : 7.0f;
+    uint8_t *xbuf = act_smem + (tid >> 2) * kXposeGroupBytes;
 
-    float2 v[2][8];
+    pdl_wait();  // X may come from, and Xq may still be read by, the previous kernel
+    pdl_launch_dependents();
+    // ---- layout A: a[j][k] = (x[8p + 32j + 2k], x[8p + 32j + 2k + 1]) of group g
+    uint4 raw[4];
     if (active) {
-        load_row_chunks(X + row * K, 0, elem0, v);
+        const __half *src = X + row * K + 128 * g + 8 * p;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) raw[j] = ld_stream_v4(src + 32 * j);
     } else {
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[h][e] = f2(0.0f);
+        for (int j = 0; j < 4; ++j) raw[j] = make_uint4(0, 0, 0, 0);
     }
     if (tid < rows) s_amax[tid] = 0u;
-    __syncthreads();
-
-    fwht_block<LOG2B>(v, lane);
-    const float2 rb = f2(rsqrt_block(LOG2B));
-    float amax = 0.0f;
+    float2 a[4][4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t ww[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            v[h][e] = __fmul2_rn(v[h][e], rb);
-            amax = fmaxf(amax, fmaxf(fabsf(v[h][e].x), fabsf(v[h][e].y)));
+        for (int k = 0; k < 4; ++k) a[j][k] = __half22float2(*reinterpret_cast<const __half2 *>(&ww[k]));
+    }
+    if (LOG2B > 1) {  // bit 1
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            bfly2(a[j][0], a[j][1]);
+            bfly2(a[j][2], a[j][3]);
         }
     }
-    const int G = reduce_width(L);
-    for (int m = 1; m < G; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
-    if (r < rows && (l & (G - 1)) == 0) atomicMax(&s_amax[r], __float_as_uint(amax));  // amax >= 0
-    __syncthreads();
-    if (active && l == 0) {
-        const float s = __fdiv_rn(__uint_as_float(s_amax[r]), qmax);
-        s_inv[r] = s == 0.0f ? 0.0f : __frcp_rn(s);
-        x_scale[row] = s;
+    if (LOG2B > 2) {  // bit 2
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            bfly2(a[j][0], a[j][2]);
+            bfly2(a[j][1], a[j][3]);
+        }
     }
-    __syncthreads();
-    if (!active) return;
-    const float2 inv = f2(s_inv[r]);
+    if (LOG2B > 5) {  // bit 5
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+        for (int k = 0; k < 4; ++k) {
+            bfly2(a[0][k], a[1][k]);
+            bfly2(a[2][k], a[3][k]);
+        }
+    }
+    if (LOG2B > 6) {  // bit 6
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[h][e] = __ffma2_rn(v[h][e], inv, f2(kRoundMagic));  // rne(x~ * inv), one rounding
-    void *out_row = BITS == 8 ? static_cast<void *>(static_cast<int8_t *>(Xq) + row * K)
-                              : static_cast<void *>(static_cast<uint8_t *>(Xq) + row * (K / 2));
-    store_codes<BITS>(out_row, elem0, v);
+        for (int k = 0; k < 4; ++k) {
+            bfly2(a[0][k], a[2][k]);
+            bfly2(a[1][k], a[3][k]);
+        }
+    }
+    // ---- A -> B: unit u = 2p + 8j + h holds elements 4u .. 4u + 3 = a[j][2h], a[j][2h+1]
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            *reinterpret_cast<float4 *>(xbuf + 16 * xpose_slot(2 * p + 8 * j + h)) =
+                make_float4(a[j][2 * h].x, a[j][2 * h].y, a[j][2 * h + 1].x, a[j][2 * h + 1].y);
+        }
+    }
+    __syncwarp();
+    // ---- layout B: b[m][c] = (x[32p + 4m + c], x[32p + 4m + c + 2])
+    float2 bv[8][2];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const float4 f = *reinterpret_cast<const float4 *>(xbuf + 16 * xpose_slot(8 * p + m));
+        bv[m][0] = make_float2(f.x, f.z);
+        bv[m][1] = make_float2(f.y, f.w);
+    }
+    if (LOG2B > 0) {  // bit 0
+#pragma unroll
+        for (int m = 0; m < 8; ++m) bfly2(bv[m][0], bv[m][1]);
+    }
+    if (LOG2B > 3) {  // bit 3
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+            if (!(m & 2)) {
+                bfly2(bv[m][0], bv[m + 2][0]);
+                bfly2(bv[m][1], bv[m + 2][1]);
+            }
+    }
+    if (LOG2B > 4) {  // bit 4
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            bfly2(bv[m][0], bv[m + 4][0]);
+            bfly2(bv[m][1], bv[m + 4][1]);
+        }
+    }
+    if (LOG2B > 7) {  // bit 7: the neighbouring 128-element group, lane l ^ 4
+        const float sgn = (lane & 4) ? -1.0f : 1.0f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float2 o;
+                o.x = __shfl_xor_sync(0xffffffffu, bv[m][c].x, 4);
+                o.y = __shfl_xor_sync(0xffffffffu, bv[m][c].y, 4);
+                bv[m][c] = __ffma2_rn(bv[m][c], f2(sgn), o);
+            }
+        }
+    }
+    // ---- row maximum of |y| (y = unnormalized rotation)
+    float amax = 0.0f;
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) amax = absmax3(amax, bv[m][c].x, bv[m][c].y);
+    const int G = reduce_width(L);
+    for (int mm = 1; mm < G; mm <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, mm));
+    // max|x~| = fp32(max|y| * rsqrt(b)) (rounding is monotone), s = fp32(that / qmax);
+    // code = rne(x~ * fp32(1/s)) with x~ = y * rsqrt(b): one factor per row
+    const float rb = rsqrt_block(LOG2B);
+    float fac1;
+    if (G == L) {
+        // the whole row lives in this warp: no block-wide step
+        if (!active) return;
+        const float sc = __fdiv_rn(__fmul_rn(amax, rb), qmax);
+        fac1 = sc == 0.0f ? 0.0f : __fmul_rn(rb, __frcp_rn(sc));
+        if (l == 0) x_scale[row] = sc;
+    } else {
+        __syncthreads();  // s_amax initialised
+        if (r < rows && (l & (G - 1)) == 0) atomicMax(&s_amax[r], __float_as_uint(amax));  // amax >= 0
+        __syncthreads();
+        if (active && l == 0) {
+            const float sc = __fdiv_rn(__fmul_rn(__uint_as_float(s_amax[r]), rb), qmax);
+            s_fac[r] = sc == 0.0f ? 0.0f : __fmul_rn(rb, __frcp_rn(sc));
+            x_scale[row] = sc;
+        }
+        __syncthreads();
+        if (!active) return;
+        fac1 = s_fac[r];
+    }
+    const float2 fac = f2(fac1);
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) bv[m][c] = __ffma2_rn(bv[m][c], fac, f2(kRoundMagic));
+    // element 4m + q of the run: q = 0 -> b[m][0].x, 1 -> b[m][1].x, 2 -> b[m][0].y, 3 -> b[m][1].y
+    uint32_t wd[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const uint32_t c01 = __byte_perm(__float_as_uint(bv[m][0].x), __float_as_uint(bv[m][1].x), 0x0040);
+        const uint32_t c23 = __byte_perm(__float_as_uint(bv[m][0].y), __float_as_uint(bv[m][1].y), 0x0040);
+        wd[m] = __byte_perm(c01, c23, 0x5410);
+    }
+    if (BITS == 8) {
+        int8_t *dst = static_cast<int8_t *>(Xq) + row * K + 128 * g + 32 * p;
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+    } else {
+        // int4 byte = code[2i] | code[2i+1] << 4
+        uint32_t nb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t even = __byte_perm(wd[2 * i], wd[2 * i + 1], 0x6420);
+            const uint32_t odd = __byte_perm(wd[2 * i], wd[2 * i + 1], 0x7531);
+            nb[i] = (even & 0x0f0f0f0fu) | ((odd & 0x0f0f0f0fu) << 4);
+        }
+        uint8_t *dst = static_cast<uint8_t *>(Xq) + row * (K / 2) + 64 * g + 16 * p;
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(nb[0], nb[1], nb[2], nb[3]);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -391,5 +539,6 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
     if (bits == 8) store_codes<8>(static_cast<int8_t *>(Wq) + row * K, elem0, q);
     else store_codes<4>(static_cast<uint8_t *>(Wq) + row * (K / 2), elem0, q);
 }
+
 
 }  // namespace convrot
