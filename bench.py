@@ -38,6 +38,24 @@ METRIC = "ConvRot W8A8/W4A4 linear TOPS and tokens/s (rotate+quant+GEMM+dequant)
 L2_BYTES = 126 * 1024 * 1024
 
 
+def replica_ids(rank: int, n_sets: int = 2) -> list:
+    """Independent input draws of one rank: weak scaling, no two ranks share a batch."""
+    return [rank * n_sets + r for r in range(n_sets)]
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's time counts (all ranks take part in the same reduction)."""
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(M: int, world: int, steps: int, elapsed_ms: float) -> float:
+    """Tokens processed by all ranks divided by the max-over-ranks elapsed time."""
+    return M * world * steps / (elapsed_ms / 1000.0)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -163,18 +181,31 @@ def run_step_linear(w, rep, stream):
 
 # ------------------------------------------------------------------------------------------ CPU oracle
 
+_ORACLE_WEIGHTS = {}
+
+
+def oracle_weights(w: wl.Workload):
+    """Inputs and oracle-converted weights of every linear (converted once, untimed,
+    as the GPU's offline conversion is)."""
+    import oracle  # the oracle is only used by the CPU baseline legs
+
+    if w.name not in _ORACLE_WEIGHTS:
+        weights = []
+        for i in range(len(w.linears)):
+            X, W, _ = wl.linear_inputs(w, i)
+            qw, sw, _ = oracle.quantize_weight(W, w.block, w.bits, oracle.CLIP_MSE)
+            weights.append((X, qw, sw))
+        _ORACLE_WEIGHTS[w.name] = weights
+    return _ORACLE_WEIGHTS[w.name]
+
+
 def time_oracle(w: wl.Workload, budget_s: float, max_rows: int | None = None):
     """Times the CPU oracle (rotate+quant, integer GEMM, dequant) on a bounded
-    sample of rows of every linear of the workload.  The offline weight
-    conversion is done first and is not timed, as on the GPU."""
-    import oracle  # the oracle is only used by this baseline leg
+    sample of rows of every linear of the workload."""
+    import oracle  # the oracle is only used by the CPU baseline legs
 
     threads = oracle.set_threads(os.cpu_count() or 1)
-    weights = []
-    for i in range(len(w.linears)):
-        X, W, _ = wl.linear_inputs(w, i)
-        qw, sw, _ = oracle.quantize_weight(W, w.block, w.bits, oracle.CLIP_MSE)
-        weights.append((X, qw, sw))
+    weights = oracle_weights(w)
 
     def run(rows):
         t0 = time.perf_counter()
@@ -251,7 +282,7 @@ def ours_arm(args, w, rank, world, local_rank):
     # offline conversion (timed once, reported separately; not part of a step)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    reps = [Replica(w, replica=rank * 2 + r, device=device) for r in range(2)]
+    reps = [Replica(w, replica=r, device=device) for r in replica_ids(rank)]
     torch.cuda.synchronize()
     setup_s = time.perf_counter() - t0
     per_set = reps[0].nbytes()
@@ -313,13 +344,10 @@ def ours_arm(args, w, rank, world, local_rank):
     cr.convrot_device_status(stream)
     clocks = clk.summary()
 
-    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
-    elapsed_ms = float(t_max.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, device)
     ms_per_step = elapsed_ms / args.steps
     tokens = w.M * world * args.steps
-    value = tokens / (elapsed_ms / 1000.0)
+    value = whole_job_tokens_per_s(w.M, world, args.steps, elapsed_ms)
 
     # end to end through the public entry point, host buffers in pinned memory
     h2d = sum(it["X"].nbytes for it in reps[0].items)
@@ -339,11 +367,10 @@ def ours_arm(args, w, rank, world, local_rank):
                 it["Yhost"].copy_(it["Y"], non_blocking=True)
         e_end.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e_start.elapsed_time(e_end)], dtype=torch.float64, device=device)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, device)
     if world > 1:
-        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.barrier()
-    e2e_value = tokens / (float(e2e_ms.item()) / 1000.0)
+    e2e_value = whole_job_tokens_per_s(w.M, world, args.steps, e2e_ms)
     cr.convrot_device_status(stream)
 
     if rank != 0:
