@@ -148,8 +148,8 @@ class Replica:
 def run_step(w, rep, stream, events=None):
     """One pass over every linear: rotate+quant kernel, then GEMM+dequant kernel.
 
-    The two kernels are launched through their own entry points (the same
-    launches convrot_linear_* makes).  With ``events`` (per linear: act start,
+    The two kernels are launched through convrot_linear_quant_act and
+    convrot_linear_gemm, the two halves of convrot_linear_*.  With ``events`` (per linear: act start,
     act end = GEMM start, GEMM end) every kernel is bracketed for per-kernel
     timing; event nodes between kernels also stop the next kernel from starting
     early, so the throughput pass runs without them.
@@ -157,17 +157,12 @@ def run_step(w, rep, stream, events=None):
     for i, it in enumerate(rep.items):
         lin = it["lin"]
         ws = it["ws"]
-        code_bytes = w.M * lin.K * w.bits // 8
-        off = (code_bytes + 255) // 256 * 256
-        xq = ws[:code_bytes].view(torch.int8 if w.bits == 8 else torch.uint8).view(w.M, -1)
-        xs = ws[off:off + 4 * w.M].view(torch.float32)
         if events is not None:
             events[i][0].record(stream)
-        cr.convrot_rotate_quant_act(it["X"], w.block, w.bits, Xq=xq, x_scale=xs, stream=stream)
+        cr.convrot_linear_quant_act(it["X"], w.block, w.bits, ws, stream=stream)
         if events is not None:
             events[i][1].record(stream)
-        gemm = cr.convrot_gemm_w8a8 if w.bits == 8 else cr.convrot_gemm_w4a4
-        gemm(xq, xs, it["Wq"], it["sw"], Y=it["Y"], stream=stream)
+        cr.convrot_linear_gemm(ws, w.M, lin.K, w.bits, it["Wq"], it["sw"], None, it["Y"], stream=stream)
         if events is not None:
             events[i][2].record(stream)
 
@@ -440,8 +435,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.workload.startswith("msweep_M"):
-        w = wl.msweep(int(args.workload[len("msweep_M"):]))
+    if args.workload.startswith("msweep"):
+        w = wl.msweep(int(args.workload.rsplit("M", 1)[1]))
     else:
         w = wl.WORKLOADS[args.workload]
 

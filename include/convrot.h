@@ -23,7 +23,7 @@
  *   X~ = X.R,  s_x[m] = max_k |X~[m,k]| / qmax,       qx = rne(X~ * (1/s_x))
  *   W~ = W.R,  s_w[n] = alpha_n max_k |W~[n,k]| / qmax, qw = clamp(rne(W~ * (1/s_w)))
  *   acc[m,n] = sum_k qx[m,k] qw[n,k]             (exact int32)
- *   Y[m,n]   = fp16( (float(acc) * s_x[m]) * s_w[n] + bias[n] )
+ *   Y[m,n]   = fp16( fma( fp32(float(acc) * s_x[m]), s_w[n], bias[n] ) )
  * qmax = 127 (int8, codes in [-127, 127]) or 7 (int4, codes in [-8, 7]).
  * Rotation and scales are fp32; every rounding is round-to-nearest-even.
  *
@@ -102,9 +102,10 @@ convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, i
 
 /*
  * Bytes of scratch the linear entry points need for M tokens of K features:
- * the activation codes (M*K for bits = 8, M*K/2 for bits = 4) and the M
- * per-token scales, each rounded up to 256 bytes.  Returns 0 for invalid
- * arguments.
+ * the activation codes, one byte per code for both widths (M*K; the W4A4
+ * linear keeps its transient int4 activation codes unpacked so that only the
+ * stored weights are widened inside the GEMM), and the M per-token scales, each
+ * rounded up to 256 bytes.  Returns 0 for invalid arguments.
  */
 size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
 
@@ -117,7 +118,8 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
  *   bias      [N] fp16 or NULL.
  *   Y         [M x N] fp16 output.
  *   workspace at least convrot_workspace_bytes(M, K, 8) bytes of device memory;
- *             its contents on return are the activation codes and scales.
+ *             its contents on return are the activation codes (int8 M x K)
+ *             followed, at the next 256-byte boundary, by the scales.
  */
 convrot_status_t convrot_linear_w8a8(const void *X, int64_t M, int64_t K, const int8_t *Wq,
                                      const float *w_scale, int64_t N, const void *bias, int block, void *Y,
@@ -133,6 +135,18 @@ convrot_status_t convrot_linear_w8a8(const void *X, int64_t M, int64_t K, const 
 convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const uint8_t *Wq,
                                      const float *w_scale, int64_t N, const void *bias, int block, void *Y,
                                      void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The two launches of convrot_linear_w8a8 / convrot_linear_w4a4, callable
+ * separately (same arguments, same workspace layout): first rotate and
+ * quantize X into the workspace, then run the integer GEMM + dequant from it.
+ * The workspace must not be reused by another linear in between.
+ */
+convrot_status_t convrot_linear_quant_act(const void *X, int64_t M, int64_t K, int block, int bits,
+                                          void *workspace, size_t workspace_bytes, void *stream);
+convrot_status_t convrot_linear_gemm(const void *workspace, size_t workspace_bytes, int64_t M, int64_t K, int bits,
+                                     const void *Wq, const float *w_scale, int64_t N, const void *bias, void *Y,
+                                     void *stream);
 
 /*
  * The integer GEMM with its dequantizing epilogue alone, on given codes (the

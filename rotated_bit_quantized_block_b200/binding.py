@@ -23,7 +23,7 @@ EXPORTED = (
     "convrot_quantize_weight", "convrot_rotate_quant_act", "convrot_workspace_bytes",
     "convrot_linear_w8a8", "convrot_linear_w4a4", "convrot_gemm_w8a8", "convrot_gemm_w4a4",
     "convrot_device_status", "convrot_status_string", "convrot_last_error", "convrot_version",
-    "convrot_linear_w8a8_noalloc",
+    "convrot_linear_w8a8_noalloc", "convrot_linear_quant_act", "convrot_linear_gemm",
 )
 
 
@@ -56,6 +56,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
             "convrot_gemm_w8a8": (i32, [P, P, i64, P, P, i64, i64, P, P, P, P]),
             "convrot_gemm_w4a4": (i32, [P, P, i64, P, P, i64, i64, P, P, P, P]),
             "convrot_linear_w8a8_noalloc": (i32, [P, i64, i64, P, P, i64, P, i32, P, P]),
+            "convrot_linear_quant_act": (i32, [P, i64, i64, i32, i32, P, sz, P]),
+            "convrot_linear_gemm": (i32, [P, sz, i64, i64, i32, P, P, i64, P, P, P]),
             "convrot_device_status": (i32, [P]),
             "convrot_status_string": (ctypes.c_char_p, [i32]),
             "convrot_last_error": (ctypes.c_char_p, []),
@@ -165,6 +167,26 @@ def convrot_linear_w8a8(X, Wq, w_scale, block, bias=None, Y=None, workspace=None
 def convrot_linear_w4a4(X, Wq, w_scale, block, bias=None, Y=None, workspace=None, stream=None):
     """Y = ConvRot W4A4 linear of X (fp16) with packed int4 weight codes Wq (N x K/2)."""
     return _linear("convrot_linear_w4a4", 4, X, Wq, w_scale, block, bias, Y, workspace, stream)
+
+
+def convrot_linear_quant_act(X, block, bits, workspace, stream=None):
+    """First launch of a linear: rotate + quantize X into the linear's workspace."""
+    _dev(X, "X")
+    M, K = X.shape
+    st = load_library().convrot_linear_quant_act(_ptr(X), M, K, block, bits, _ptr(workspace),
+                                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st)
+
+
+def convrot_linear_gemm(workspace, M, K, bits, Wq, w_scale, bias=None, Y=None, stream=None):
+    """Second launch of a linear: integer GEMM + dequant from the workspace."""
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=Wq.device)
+    st = load_library().convrot_linear_gemm(_ptr(workspace), workspace.numel() * workspace.element_size(), M, K,
+                                            bits, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y), _stream(stream))
+    _check(st)
+    return Y
 
 
 def _gemm(fn_name, Xq, x_scale, Wq, w_scale, K, bias, Y, acc_out, stream):

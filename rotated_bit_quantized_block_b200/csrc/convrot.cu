@@ -203,9 +203,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int LOG2B, int BITS>
+template <int LOG2B, int BITS, bool PACKED>
 void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms, int dev) {
-    auto kern = convrot::act_rotate_quant_kernel<LOG2B, BITS>;
+    auto kern = convrot::act_rotate_quant_kernel<LOG2B, BITS, PACKED>;
     {
         static bool configured[kMaxDevices];
         static std::mutex mu;
@@ -224,19 +224,19 @@ void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaSt
                static_cast<const __half *>(X), M, static_cast<int>(K), R, Xq, xs);
 }
 
-template <int BITS>
+template <int BITS, bool PACKED>
 void dispatch_act(int log2b, const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms,
                   int dev) {
     switch (log2b) {
-        case 0: launch_act<0, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 1: launch_act<1, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 2: launch_act<2, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 3: launch_act<3, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 4: launch_act<4, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 5: launch_act<5, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 6: launch_act<6, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 7: launch_act<7, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
-        default: launch_act<8, BITS>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 0: launch_act<0, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 1: launch_act<1, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 2: launch_act<2, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 3: launch_act<3, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 4: launch_act<4, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 5: launch_act<5, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 6: launch_act<6, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 7: launch_act<7, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
+        default: launch_act<8, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
     }
 }
 
@@ -250,11 +250,13 @@ void launch_weight(const void *W, int dtype, int64_t N, int64_t K, int bits, int
         W, dtype, N, static_cast<int>(K), R, bits, clip, Wq, ws);
 }
 
-convrot_status_t rotate_quant_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, void *Xq,
-                                       float *x_scale, cudaStream_t st, int sms, int dev) {
+// packed: int4 codes two per byte (bits = 4 only); otherwise one byte per code.
+convrot_status_t rotate_quant_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, bool packed,
+                                       void *Xq, float *x_scale, cudaStream_t st, int sms, int dev) {
     const int log2b = ilog2(block);
-    if (bits == 8) dispatch_act<8>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
-    else dispatch_act<4>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
+    if (bits == 8) dispatch_act<8, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
+    else if (packed) dispatch_act<4, true>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
+    else dispatch_act<4, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
     return launch_status("act_rotate_quant");
 }
 
@@ -276,11 +278,15 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *A, const
         }
     }
     CUtensorMap ta, tb, ty;
-    const int64_t row_bytes = Cfg::W4 ? K / 2 : K;
-    const int box_bytes = Cfg::W4 ? Cfg::BK / 2 : Cfg::BK;
-    const CUtensorMapSwizzle sw_in = Cfg::W4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
-    CR_TRY(make_map(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, row_bytes, Cfg::BM, box_bytes, sw_in));
-    CR_TRY(make_map(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, row_bytes, Cfg::BN, box_bytes, sw_in));
+    // int8 operands: 128-byte boxes with the 128B swizzle the MMA reads; packed
+    // int4 operands: 64-byte boxes of dense rows for the converters
+    const auto op_map = [&](CUtensorMap *m, const void *base, int64_t rows, int box_rows, bool packed) {
+        return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, packed ? K / 2 : K, box_rows,
+                        packed ? Cfg::BK / 2 : Cfg::BK,
+                        packed ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
+    };
+    CR_TRY(op_map(&ta, A, M, Cfg::BM, Cfg::A4));
+    CR_TRY(op_map(&tb, B, N, Cfg::BN, Cfg::B4));
     CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, Cfg::CHUNK, CU_TENSOR_MAP_SWIZZLE_128B));
     const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
     const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
@@ -291,15 +297,17 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *A, const
 }
 
 // Picks the tile width: the widest tile that still gives every SM work.
-template <bool W4>
+// A4 / B4: activation / weight operand packed int4.
+template <bool A4, bool B4>
 convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *A, const void *B, int64_t M, int64_t N,
                              int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
                              int32_t *acc_out, cudaStream_t st) {
     const int64_t tiles_m = (M + 127) / 128;
     const int64_t tiles_256 = tiles_m * ((N + 255) / 256);
     if (N >= 256 && tiles_256 >= info->sms)
-        return launch_gemm_cfg<convrot::GemmCfg<256, W4>>(info, dev, A, B, M, N, K, sx, sw, bias, Y, acc_out, st);
-    return launch_gemm_cfg<convrot::GemmCfg<128, W4>>(info, dev, A, B, M, N, K, sx, sw, bias, Y, acc_out, st);
+        return launch_gemm_cfg<convrot::GemmCfg<256, A4, B4>>(info, dev, A, B, M, N, K, sx, sw, bias, Y, acc_out,
+                                                              st);
+    return launch_gemm_cfg<convrot::GemmCfg<128, A4, B4>>(info, dev, A, B, M, N, K, sx, sw, bias, Y, acc_out, st);
 }
 
 convrot_status_t check_gemm_args(const void *Xq, const float *xs, int64_t M, const void *Wq, const float *ws,
@@ -345,7 +353,9 @@ int convrot_version(void) { return kVersion; }
 
 size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits) {
     if (M < 0 || K <= 0 || (bits != 8 && bits != 4)) return 0;
-    const size_t codes = static_cast<size_t>(M) * static_cast<size_t>(K) * static_cast<size_t>(bits) / 8;
+    // the linears keep one byte per activation code (int4 codes are widened
+    // once here instead of in every GEMM tile that reads them)
+    const size_t codes = static_cast<size_t>(M) * static_cast<size_t>(K);
     return round256(codes) + round256(static_cast<size_t>(M) * 4);
 }
 
@@ -392,34 +402,93 @@ convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, i
     int dev;
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
-    return rotate_quant_act_impl(X, M, K, block, bits, Xq, x_scale, static_cast<cudaStream_t>(stream), info->sms, dev);
+    return rotate_quant_act_impl(X, M, K, block, bits, bits == 4, Xq, x_scale, static_cast<cudaStream_t>(stream),
+                                 info->sms, dev);
+}
+
+// Workspace layout of the linears: activation codes (one byte each) then, at
+// the next 256-byte boundary, the per-token scales.
+static void workspace_parts(void *workspace, int64_t M, int64_t K, void **xq, float **xs) {
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    *xq = ws;
+    *xs = reinterpret_cast<float *>(ws + round256(static_cast<size_t>(M) * K));
+}
+
+static convrot_status_t check_linear_shape(int64_t M, int64_t K, int block, int bits, int64_t N) {
+    CR_TRY(check_shape(M, K, block, "M"));
+    CR_TRY(check_bits(bits));
+    CR_REQUIRE(N >= 0 && N < (int64_t(1) << 31) && N % 8 == 0, CONVROT_ERR_INVALID_ARG,
+               "N = %lld must be a multiple of 8 in [0, 2^31)", static_cast<long long>(N));
+    return ok();
+}
+
+static convrot_status_t check_workspace(const void *workspace, size_t workspace_bytes, int64_t M, int64_t K,
+                                        int bits) {
+    const size_t need = convrot_workspace_bytes(M, K, bits);
+    CR_REQUIRE(workspace != nullptr && workspace_bytes >= need, CONVROT_ERR_WORKSPACE,
+               "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+    CR_REQUIRE(aligned(workspace, 16), CONVROT_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+    return ok();
+}
+
+static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, void *workspace,
+                                        size_t workspace_bytes, cudaStream_t st) {
+    CR_REQUIRE(X != nullptr, CONVROT_ERR_INVALID_ARG, "null pointer argument");
+    CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
+    CR_TRY(check_workspace(workspace, workspace_bytes, M, K, bits));
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    void *xq;
+    float *xs;
+    workspace_parts(workspace, M, K, &xq, &xs);
+    return rotate_quant_act_impl(X, M, K, block, bits, false, xq, xs, st, info->sms, dev);
+}
+
+static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace_bytes, int64_t M, int64_t K,
+                                         int bits, const void *Wq, const float *w_scale, int64_t N,
+                                         const void *bias, void *Y, cudaStream_t st) {
+    CR_TRY(check_workspace(workspace, workspace_bytes, M, K, bits));
+    void *xq;
+    float *xs;
+    workspace_parts(const_cast<void *>(workspace), M, K, &xq, &xs);
+    CR_TRY(check_gemm_args(xq, xs, M, Wq, w_scale, N, K, bias, Y));
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    if (bits == 8) return launch_gemm<false, false>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
+    return launch_gemm<false, true>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
 }
 
 static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t K, const void *Wq,
                                     const float *w_scale, int64_t N, const void *bias, int block, void *Y,
                                     void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error.clear();
-    CR_TRY(check_shape(M, K, block, "M"));
-    CR_REQUIRE(N >= 0 && N < (int64_t(1) << 31) && N % 8 == 0, CONVROT_ERR_INVALID_ARG,
-               "N = %lld must be a multiple of 8 in [0, 2^31)", static_cast<long long>(N));
+    CR_TRY(check_linear_shape(M, K, block, bits, N));
     if (M == 0 || N == 0) return ok();
     CR_REQUIRE(X && Wq && w_scale && Y, CONVROT_ERR_INVALID_ARG, "null pointer argument");
-    const size_t need = convrot_workspace_bytes(M, K, bits);
-    CR_REQUIRE(workspace != nullptr && workspace_bytes >= need, CONVROT_ERR_WORKSPACE,
-               "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
-    CR_REQUIRE(aligned(workspace, 16), CONVROT_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
-    CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    void *xq = ws;
-    float *xs = reinterpret_cast<float *>(ws + round256(static_cast<size_t>(M) * K * bits / 8));
-    CR_TRY(check_gemm_args(xq, xs, M, Wq, w_scale, N, K, bias, Y));
-    int dev;
-    DeviceInfo *info;
-    CR_TRY(current_device(&dev, &info));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    CR_TRY(rotate_quant_act_impl(X, M, K, block, bits, xq, xs, st, info->sms, dev));
-    if (bits == 8) return launch_gemm<false>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
-    return launch_gemm<true>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
+    CR_TRY(linear_act_impl(X, M, K, block, bits, workspace, workspace_bytes, st));
+    return linear_gemm_impl(workspace, workspace_bytes, M, K, bits, Wq, w_scale, N, bias, Y, st);
+}
+
+convrot_status_t convrot_linear_quant_act(const void *X, int64_t M, int64_t K, int block, int bits, void *workspace,
+                                          size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    CR_TRY(check_shape(M, K, block, "M"));
+    CR_TRY(check_bits(bits));
+    if (M == 0) return ok();
+    return linear_act_impl(X, M, K, block, bits, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+convrot_status_t convrot_linear_gemm(const void *workspace, size_t workspace_bytes, int64_t M, int64_t K, int bits,
+                                     const void *Wq, const float *w_scale, int64_t N, const void *bias, void *Y,
+                                     void *stream) {
+    g_last_error.clear();
+    CR_TRY(check_linear_shape(M, K, 1, bits, N));
+    if (M == 0 || N == 0) return ok();
+    return linear_gemm_impl(workspace, workspace_bytes, M, K, bits, Wq, w_scale, N, bias, Y,
+                            static_cast<cudaStream_t>(stream));
 }
 
 convrot_status_t convrot_linear_w8a8(const void *X, int64_t M, int64_t K, const int8_t *Wq, const float *w_scale,
@@ -445,8 +514,8 @@ static convrot_status_t gemm_impl(bool w4, const void *Xq, const float *x_scale,
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (w4) return launch_gemm<true>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st);
-    return launch_gemm<false>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st);
+    if (w4) return launch_gemm<true, true>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st);
+    return launch_gemm<false, false>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st);
 }
 
 convrot_status_t convrot_gemm_w8a8(const int8_t *Xq, const float *x_scale, int64_t M, const int8_t *Wq,

@@ -26,21 +26,31 @@
 
 namespace convrot {
 
-template <int BN_, bool W4_>
+// A4 / B4: the activation / weight operand arrives as packed int4 (two codes
+// per byte) and is widened in shared memory; otherwise it is int8 loaded by TMA
+// straight into the MMA ring.  Widened bytes hold 16 * code, so the
+// accumulator carries a factor 16 per widened operand (ACC_SHIFT undoes it).
+template <int BN_, bool A4_, bool B4_>
 struct GemmCfg {
     static constexpr int BM = 128;
     static constexpr int BN = BN_;
     static constexpr int BK = 128;  // K elements per stage (= bytes of one int8 row segment)
-    static constexpr bool W4 = W4_;
+    static constexpr bool A4 = A4_;
+    static constexpr bool B4 = B4_;
+    static constexpr bool W4 = A4 || B4;  // some operand is widened by converter warps
+    static constexpr int ACC_SHIFT = (A4 ? 4 : 0) + (B4 ? 4 : 0);
     static constexpr int A_BYTES = BM * BK;
     static constexpr int B_BYTES = BN * BK;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    // MMA ring depth and (W4A4) packed ring depth
-    static constexpr int STAGES = W4 ? (BN == 256 ? 2 : 3) : (BN == 256 ? 4 : 6);
-    static constexpr int PSTAGES = W4 ? (BN == 256 ? 3 : 4) : 0;
-    static constexpr int PA_BYTES = A_BYTES / 2;
+    // MMA ring depth and packed ring depth
+    static constexpr int STAGES = !W4 ? (BN == 256 ? 4 : 6) : A4 ? (BN == 256 ? 2 : 3) : (BN == 256 ? 3 : 4);
+    static constexpr int PSTAGES = !W4 ? 0 : (BN == 256 ? 3 : 4);
+    static constexpr int PA_BYTES = A4 ? A_BYTES / 2 : 0;
     static constexpr int PB_BYTES = B_BYTES / 2;
     static constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
+    static constexpr int CONV_ROWS = (A4 ? BM : 0) + BN;  // rows widened per stage
+    // arrivals completing an MMA stage: the producer (A bytes by TMA) and/or the converters
+    static constexpr int FULL_COUNT = !W4 ? 1 : (A4 ? 128 : 129);
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int EPI_WARPS = 8;           // two per TMEM lane quarter, each half of the columns
     static constexpr int EPI_COLS = BN / 2;       // columns per epilogue warp
@@ -77,7 +87,7 @@ __device__ __forceinline__ uint4 widen_int4x16(uint2 p) {
 // Dequantizes 8 accumulators of one row: fp16(fma(fp32(float(acc) * sx), sw[c], bias[c]))
 // (the final multiply-add is one explicit fused operation, so it rounds once).
 // sw_s / bias_s point at the tile's scales staged in shared memory.
-template <bool W4>
+template <int SHIFT>
 __device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const float *sw_s, const __half *bias_s,
                                           int32_t *acc_vals) {
     const float4 w0 = *reinterpret_cast<const float4 *>(sw_s);
@@ -88,8 +98,8 @@ __device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const fl
     uint32_t out[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int32_t a0 = W4 ? (static_cast<int32_t>(r[2 * i]) >> 8) : static_cast<int32_t>(r[2 * i]);
-        const int32_t a1 = W4 ? (static_cast<int32_t>(r[2 * i + 1]) >> 8) : static_cast<int32_t>(r[2 * i + 1]);
+        const int32_t a0 = static_cast<int32_t>(r[2 * i]) >> SHIFT;
+        const int32_t a1 = static_cast<int32_t>(r[2 * i + 1]) >> SHIFT;
         acc_vals[2 * i] = a0;
         acc_vals[2 * i + 1] = a1;
         const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&bw[i]));
@@ -136,7 +146,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&full[i], Cfg::W4 ? 128 : 1);
+            mbar_init(&full[i], Cfg::FULL_COUNT);
             mbar_init(&empty[i], 1);
         }
         for (int i = 0; i < PSTAGES; ++i) {
@@ -172,44 +182,60 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const int nst = Cfg::W4 ? PSTAGES : STAGES;
-            uint64_t *ld_full = Cfg::W4 ? pfull : full;
-            uint64_t *ld_empty = Cfg::W4 ? pempty : empty;
-            uint32_t last_parity[(Cfg::W4 ? PSTAGES : STAGES)];
-            bool filled[(Cfg::W4 ? PSTAGES : STAGES)];
-            for (int i = 0; i < nst; ++i) filled[i] = false;
-            int s = 0;
-            uint32_t ph = 0;
+            // MMA ring (s, ph): int8 operands loaded straight by TMA; packed ring
+            // (ps, pph): int4 operands for the converters
+            int s = 0, ps = 0;
+            uint32_t ph = 0, pph = 0;
+            uint32_t last_parity[STAGES > PSTAGES ? STAGES : PSTAGES];
+            uint32_t plast_parity[PSTAGES > 0 ? PSTAGES : 1];
+            bool filled[STAGES > PSTAGES ? STAGES : PSTAGES], pfilled[PSTAGES > 0 ? PSTAGES : 1];
+            for (int i = 0; i < STAGES; ++i) filled[i] = false;
+            for (int i = 0; i < PSTAGES; ++i) pfilled[i] = false;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
                 const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(&ld_empty[s], ph ^ 1, abort)) {
-                        ok = false;
-                        break;
+                    if (!Cfg::A4) {
+                        if (!mbar_wait(&empty[s], ph ^ 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *dst = ring + s * Cfg::STAGE_BYTES;
+                        const uint32_t bytes = Cfg::B4 ? Cfg::A_BYTES : Cfg::STAGE_BYTES;
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                        tma_load_2d(dst, &tmA, &full[s], kb * Cfg::BK, tm * BM);
+                        if (!Cfg::B4) tma_load_2d(dst + Cfg::A_BYTES, &tmB, &full[s], kb * Cfg::BK, tn * BN);
+                        filled[s] = true;
+                        last_parity[s] = ph;
+                        if (++s == STAGES) {
+                            s = 0;
+                            ph ^= 1;
+                        }
                     }
                     if (Cfg::W4) {
-                        uint8_t *dst = pring + s * Cfg::PSTAGE_BYTES;
-                        mbar_arrive_expect_tx(&ld_full[s], Cfg::PSTAGE_BYTES);
-                        tma_load_2d(dst, &tmA, &ld_full[s], kb * (Cfg::BK / 2), tm * BM);
-                        tma_load_2d(dst + Cfg::PA_BYTES, &tmB, &ld_full[s], kb * (Cfg::BK / 2), tn * BN);
-                    } else {
-                        uint8_t *dst = ring + s * Cfg::STAGE_BYTES;
-                        mbar_arrive_expect_tx(&ld_full[s], Cfg::STAGE_BYTES);
-                        tma_load_2d(dst, &tmA, &ld_full[s], kb * Cfg::BK, tm * BM);
-                        tma_load_2d(dst + Cfg::A_BYTES, &tmB, &ld_full[s], kb * Cfg::BK, tn * BN);
-                    }
-                    filled[s] = true;
-                    last_parity[s] = ph;
-                    if (++s == nst) {
-                        s = 0;
-                        ph ^= 1;
+                        if (!mbar_wait(&pempty[ps], pph ^ 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *dst = pring + ps * Cfg::PSTAGE_BYTES;
+                        mbar_arrive_expect_tx(&pfull[ps], Cfg::PSTAGE_BYTES);
+                        if (Cfg::A4) tma_load_2d(dst, &tmA, &pfull[ps], kb * (Cfg::BK / 2), tm * BM);
+                        tma_load_2d(dst + Cfg::PA_BYTES, &tmB, &pfull[ps], kb * (Cfg::BK / 2), tn * BN);
+                        pfilled[ps] = true;
+                        plast_parity[ps] = pph;
+                        if (++ps == PSTAGES) {
+                            ps = 0;
+                            pph ^= 1;
+                        }
                     }
                 }
             }
             // no bulk copy may still be writing shared memory when the CTA exits
-            for (int i = 0; i < nst; ++i)
-                if (filled[i]) mbar_wait_drain(&ld_full[i], last_parity[i]);
+            // (an MMA stage also waits for its converters when B is widened)
+            for (int i = 0; i < STAGES; ++i)
+                if (filled[i]) mbar_wait_drain(&full[i], last_parity[i]);
+            for (int i = 0; i < PSTAGES; ++i)
+                if (pfilled[i]) mbar_wait_drain(&pfull[i], plast_parity[i]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -317,7 +343,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     int32_t av[8];
                     uint4 v = make_uint4(0, 0, 0, 0);
                     if (row_ok && col0 + 8 * g < N) {
-                        v = dequant8<Cfg::W4>(r[g >> 2] + 8 * (g & 3), sxm, sw_s + col_local + 8 * g,
+                        v = dequant8<Cfg::ACC_SHIFT>(r[g >> 2] + 8 * (g & 3), sxm, sw_s + col_local + 8 * g,
                                               bias_s + col_local + 8 * g, av);
                         if (acc_out != nullptr) {
                             int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0 + 8 * g);
@@ -351,11 +377,12 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     break;
                 }
                 const uint8_t *src = pring + ps * Cfg::PSTAGE_BYTES;
-                uint8_t *dst = ring + us * Cfg::STAGE_BYTES;
-                constexpr int PIECES = (BM + BN) * (Cfg::BK / 16);  // 16 codes per piece
+                // widened rows: A (if packed) then B, in the MMA ring's layout
+                uint8_t *dst = ring + us * Cfg::STAGE_BYTES + (Cfg::A4 ? 0 : Cfg::A_BYTES);
+                constexpr int PIECES = Cfg::CONV_ROWS * (Cfg::BK / 16);  // 16 codes per piece
 #pragma unroll 4
                 for (int idx = ct; idx < PIECES; idx += 128) {
-                    const int rr = idx >> 3, piece = idx & 7;  // row over A then B; 16-byte chunk in the row
+                    const int rr = idx >> 3, piece = idx & 7;  // widened row; 16-byte chunk in the row
                     const uint2 p = *reinterpret_cast<const uint2 *>(src + rr * 64 + piece * 8);
                     *reinterpret_cast<uint4 *>(dst + rr * 128 + ((piece ^ (rr & 7)) << 4)) = widen_int4x16(p);
                 }

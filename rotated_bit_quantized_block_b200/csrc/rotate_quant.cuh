@@ -239,7 +239,9 @@ __device__ __forceinline__ float absmax3(float m, float x, float y) {
 // Dynamic shared memory of the activation kernel for a block of `threads`.
 __host__ __device__ constexpr int act_smem_bytes(int threads) { return (threads / 4) * kXposeGroupBytes; }
 
-template <int LOG2B, int BITS>
+// BITS fixes the code range (8: [-127, 127], 4: [-8, 7]); PACKED stores int4
+// codes two per byte, otherwise every code takes one byte.
+template <int LOG2B, int BITS, bool PACKED>
 __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__restrict__ X, int64_t M, int K,
                                                                 int rows, void *__restrict__ Xq,
                                                                 float *__restrict__ x_scale) {
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
         const uint32_t c23 = __byte_perm(__float_as_uint(bv[m][0].y), __float_as_uint(bv[m][1].y), 0x0040);
         wd[m] = __byte_perm(c01, c23, 0x5410);
     }
-    if (BITS == 8) {
+    if (!PACKED) {
         int8_t *dst = static_cast<int8_t *>(Xq) + row * K + 128 * g + 32 * p;
         *reinterpret_cast<uint4 *>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);

@@ -54,7 +54,7 @@ def test_status_strings(lib):
 
 def test_workspace_bytes(lib):
     assert lib.convrot_workspace_bytes(5184, 1024, 8) == 5184 * 1024 + ((5184 * 4 + 255) // 256) * 256
-    assert lib.convrot_workspace_bytes(5184, 1024, 4) == 5184 * 512 + ((5184 * 4 + 255) // 256) * 256
+    assert lib.convrot_workspace_bytes(5184, 1024, 4) == 5184 * 1024 + ((5184 * 4 + 255) // 256) * 256
     assert lib.convrot_workspace_bytes(3, 128, 8) == 512 + 256
     assert lib.convrot_workspace_bytes(-1, 128, 8) == 0
     assert lib.convrot_workspace_bytes(4, 128, 5) == 0

@@ -294,3 +294,17 @@ def test_linear_msweep(M):
     rows = None if M <= 128 else np.linspace(0, M - 1, 24).astype(int)
     y, yr, _ = linear_pair(w, 0, sample=rows)
     assert rel_fro(y, yr) <= REL_FRO
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_linear_two_stage_entry_points_equal_the_linear(bits):
+    w = wl.WORKLOADS["vit_l_w8a8"]
+    X, W, bias = wl.linear_inputs(w, 3, M=700, with_bias=True)
+    Xd, Wd, bd = dev(X), dev(W), dev(bias)
+    Wq, sw = cr.convrot_quantize_weight(Wd, w.block, bits, cr.CLIP_MSE)
+    ws = torch.empty(cr.convrot_workspace_bytes(700, W.shape[1], bits), dtype=torch.uint8, device="cuda")
+    fn = cr.convrot_linear_w8a8 if bits == 8 else cr.convrot_linear_w4a4
+    y1 = host(fn(Xd, Wq, sw, w.block, bias=bd, workspace=ws))
+    cr.convrot_linear_quant_act(Xd, w.block, bits, ws)
+    y2 = host(cr.convrot_linear_gemm(ws, 700, W.shape[1], bits, Wq, sw, bias=bd))
+    assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
