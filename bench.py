@@ -132,7 +132,7 @@ class Replica:
             Xd = torch.from_numpy(X).to(device)
             Wd = torch.from_numpy(W).to(device)
             Wq, sw = cr.convrot_quantize_weight(Wd, w.block, w.bits, cr.CLIP_MSE)
-            need = cr.convrot_workspace_bytes(w.M, lin.K, w.bits)
+            need = cr.convrot_linear_workspace_bytes(w.M, lin.K, lin.N, w.bits)
             self.items.append({
                 "lin": lin, "X": Xd, "Xhost": torch.from_numpy(X).pin_memory(), "Wq": Wq, "sw": sw,
                 "Y": torch.empty((w.M, lin.N), dtype=torch.float16, device=device),

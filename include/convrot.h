@@ -110,6 +110,20 @@ convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, i
 size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
 
 /*
+ * Workspace size that also lets the linear split the K loop of its GEMM across
+ * SMs.  For few tokens (M <= 256) the GEMM runs feature-major (128 output
+ * features per tile) and has too few tiles to fill the GPU; with this
+ * workspace the K slices of a tile run on separate SMs and add their int32
+ * partials into an M x N buffer.  Size: convrot_workspace_bytes(M, K, bits)
+ * plus 2 KB of split-K counters plus that buffer (rounded up to 256 bytes)
+ * when the GEMM will split.  The activation half of the linear zeroes what
+ * follows the scales (the counters and the buffer); the GEMM half leaves both
+ * zeroed again.  With only the minimum workspace the linears never split.
+ * Depends on the current device's SM count.  Returns 0 for invalid arguments.
+ */
+size_t convrot_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
+
+/*
  * W8A8 ConvRot linear (civarchive ConvRot release, "The INT8 file uses W8A8
  * operations"): Y = dequant( int8(rotate(X)) . Wq^T ) + bias.
  *   X         [M x K] fp16 activations (not yet rotated).
@@ -117,9 +131,10 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
  *   w_scale   [N] fp32 per-output-row scales.
  *   bias      [N] fp16 or NULL.
  *   Y         [M x N] fp16 output.
- *   workspace at least convrot_workspace_bytes(M, K, 8) bytes of device memory;
- *             its contents on return are the activation codes (int8 M x K)
- *             followed, at the next 256-byte boundary, by the scales.
+ *   workspace at least convrot_workspace_bytes(M, K, 8) bytes of device memory
+ *             (convrot_linear_workspace_bytes(M, K, N, 8) enables split-K); on
+ *             return it holds the activation codes (int8 M x K) followed, at the
+ *             next 256-byte boundary, by the scales.
  */
 convrot_status_t convrot_linear_w8a8(const void *X, int64_t M, int64_t K, const int8_t *Wq,
                                      const float *w_scale, int64_t N, const void *bias, int block, void *Y,
@@ -140,7 +155,10 @@ convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const 
  * The two launches of convrot_linear_w8a8 / convrot_linear_w4a4, callable
  * separately (same arguments, same workspace layout): first rotate and
  * quantize X into the workspace, then run the integer GEMM + dequant from it.
- * The workspace must not be reused by another linear in between.
+ * The workspace must not be reused by another linear in between.  Not knowing
+ * N, convrot_linear_quant_act zeroes everything after the scales (for M <= 256
+ * at most the split state of a GEMM with N <= 32768; for larger M only the
+ * counters).
  */
 convrot_status_t convrot_linear_quant_act(const void *X, int64_t M, int64_t K, int block, int bits,
                                           void *workspace, size_t workspace_bytes, void *stream);

@@ -24,6 +24,7 @@ EXPORTED = (
     "convrot_linear_w8a8", "convrot_linear_w4a4", "convrot_gemm_w8a8", "convrot_gemm_w4a4",
     "convrot_device_status", "convrot_status_string", "convrot_last_error", "convrot_version",
     "convrot_linear_w8a8_noalloc", "convrot_linear_quant_act", "convrot_linear_gemm",
+    "convrot_linear_workspace_bytes",
 )
 
 
@@ -51,6 +52,7 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
             "convrot_quantize_weight": (i32, [P, i32, i64, i64, i32, i32, i32, P, P, P]),
             "convrot_rotate_quant_act": (i32, [P, i64, i64, i32, i32, P, P, P]),
             "convrot_workspace_bytes": (sz, [i64, i64, i32]),
+            "convrot_linear_workspace_bytes": (sz, [i64, i64, i64, i32]),
             "convrot_linear_w8a8": (i32, [P, i64, i64, P, P, i64, P, i32, P, P, sz, P]),
             "convrot_linear_w4a4": (i32, [P, i64, i64, P, P, i64, P, i32, P, P, sz, P]),
             "convrot_gemm_w8a8": (i32, [P, P, i64, P, P, i64, i64, P, P, P, P]),
@@ -143,14 +145,19 @@ def convrot_workspace_bytes(M: int, K: int, bits: int) -> int:
     return int(load_library().convrot_workspace_bytes(M, K, bits))
 
 
+def convrot_linear_workspace_bytes(M: int, K: int, N: int, bits: int) -> int:
+    """Workspace that also enables split-K in the linear's GEMM."""
+    return int(load_library().convrot_linear_workspace_bytes(M, K, N, bits))
+
+
 def _linear(fn_name, bits, X, Wq, w_scale, block, bias, Y, workspace, stream):
     _dev(X, "X")
     M, K = X.shape
     N = Wq.shape[0]
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
-    need = convrot_workspace_bytes(M, K, bits)
     if workspace is None:
+        need = convrot_linear_workspace_bytes(M, K, N, bits)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
     fn = getattr(load_library(), fn_name)
     st = fn(_ptr(X), M, K, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), block, _ptr(Y), _ptr(workspace),
@@ -246,7 +253,7 @@ class QuantizedLinear:
         self._ws = None
 
     def workspace(self, M: int, device) -> torch.Tensor:
-        need = convrot_workspace_bytes(M, self.K, self.bits)
+        need = convrot_linear_workspace_bytes(M, self.K, self.N, self.bits)
         if self._ws is None or self._ws.numel() < need or self._ws.device != device:
             self._ws = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
         return self._ws

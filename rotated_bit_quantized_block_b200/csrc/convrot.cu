@@ -204,7 +204,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 template <int LOG2B, int BITS, bool PACKED>
-void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms, int dev) {
+void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms, int dev,
+                uint4 *zero16, int64_t n_zero16) {
     auto kern = convrot::act_rotate_quant_kernel<LOG2B, BITS, PACKED>;
     {
         static bool configured[kMaxDevices];
@@ -221,22 +222,22 @@ void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaSt
     act_geometry(kern, sms, M, K, &R, &T);
     const int64_t grid = (M + R - 1) / R;
     launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(T), static_cast<size_t>(convrot::act_smem_bytes(T)), st,
-               static_cast<const __half *>(X), M, static_cast<int>(K), R, Xq, xs);
+               static_cast<const __half *>(X), M, static_cast<int>(K), R, Xq, xs, zero16, n_zero16);
 }
 
 template <int BITS, bool PACKED>
 void dispatch_act(int log2b, const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms,
-                  int dev) {
+                  int dev, uint4 *zw, int64_t nzw) {
     switch (log2b) {
-        case 0: launch_act<0, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 1: launch_act<1, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 2: launch_act<2, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 3: launch_act<3, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 4: launch_act<4, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 5: launch_act<5, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 6: launch_act<6, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
-        case 7: launch_act<7, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
-        default: launch_act<8, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev); break;
+        case 0: launch_act<0, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
+        case 1: launch_act<1, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
+        case 2: launch_act<2, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
+        case 3: launch_act<3, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
+        case 4: launch_act<4, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
+        case 5: launch_act<5, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
+        case 6: launch_act<6, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
+        case 7: launch_act<7, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
+        default: launch_act<8, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
     }
 }
 
@@ -252,20 +253,67 @@ void launch_weight(const void *W, int dtype, int64_t N, int64_t K, int bits, int
 
 // packed: int4 codes two per byte (bits = 4 only); otherwise one byte per code.
 convrot_status_t rotate_quant_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, bool packed,
-                                       void *Xq, float *x_scale, cudaStream_t st, int sms, int dev) {
+                                       void *Xq, float *x_scale, cudaStream_t st, int sms, int dev,
+                                       uint4 *zero16 = nullptr, int64_t n_zero16 = 0) {
     const int log2b = ilog2(block);
-    if (bits == 8) dispatch_act<8, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
-    else if (packed) dispatch_act<4, true>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
-    else dispatch_act<4, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev);
+    if (bits == 8) dispatch_act<8, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev, zero16, n_zero16);
+    else if (packed) dispatch_act<4, true>(log2b, X, M, K, Xq, x_scale, st, sms, dev, zero16, n_zero16);
+    else dispatch_act<4, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev, zero16, n_zero16);
     return launch_status("act_rotate_quant");
 }
 
 // ---------------------------------------------------------------- GEMM launch
 
+// GEMM launch plan: operand order, tile width and K split.
+struct GemmPlan {
+    bool swap = false;  // feature-major (weights on the MMA's 128-row side)
+    int bn = 256;       // MMA N: output features (token-major) or tokens (feature-major)
+    int splits = 1;
+    int64_t tiles = 0;
+};
+
+constexpr int kMaxSplitTiles = 512;              // split-K counters in a linear's workspace
+constexpr size_t kCounterBytes = kMaxSplitTiles * 4;
+constexpr int64_t kSwapMaxTokens = 256;          // feature-major below this many tokens
+constexpr int64_t kMaxSplitFeatures = 32768;     // split K only for N up to this
+
+// Few tokens: feature-major tiles (128 features x 32 / 128 / 256 tokens), K
+// split so that the tiles x splits units cover the SMs (at most 8 slices, each
+// at least two 128-deep K steps).  Otherwise token-major 128 x 256 tiles,
+// narrowed to 128 when 256-wide tiles would leave more than half the SMs idle.
+GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split) {
+    GemmPlan p;
+    if (M <= kSwapMaxTokens) {
+        p.swap = true;
+        p.bn = M <= 32 ? 32 : (M <= 128 ? 128 : 256);
+        p.tiles = ((N + 127) / 128) * ((M + p.bn - 1) / p.bn);
+        if (allow_split && p.tiles > 0 && p.tiles <= kMaxSplitTiles && N <= kMaxSplitFeatures) {
+            int64_t s = sms / p.tiles;
+            if (s > 8) s = 8;
+            if (s > K / 256) s = K / 256;
+            if (s >= 2) p.splits = static_cast<int>(s);
+        }
+        return p;
+    }
+    const int64_t tiles_m = (M + 127) / 128;
+    const int64_t tiles_256 = tiles_m * ((N + 255) / 256);
+    p.bn = (N >= 256 && 2 * tiles_256 > sms) ? 256 : 128;
+    p.tiles = tiles_m * ((N + p.bn - 1) / p.bn);
+    return p;
+}
+
+// int32 M x N sum buffer of a split feature-major GEMM.
+size_t split_buffer_bytes(const GemmPlan &p, int64_t M, int64_t N) {
+    return p.splits > 1 ? round256(static_cast<size_t>(M) * N * 4) : 0;
+}
+
+// Xc: activation codes (M x K), Wc: weight codes (N x K); A4 / B4 of Cfg refer
+// to the MMA's operands (token-major: A = activations; feature-major: A = weights).
 template <class Cfg>
-convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *A, const void *B, int64_t M, int64_t N,
+convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, const void *Wc, int64_t M, int64_t N,
                                  int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
-                                 int32_t *acc_out, cudaStream_t st) {
+                                 int32_t *acc_out, cudaStream_t st, int splits, int32_t *acc_buf,
+                                 unsigned int *counters) {
     {
         static std::mutex mu;
         static bool done[kMaxDevices] = {};
@@ -285,29 +333,41 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *A, const
                         packed ? Cfg::BK / 2 : Cfg::BK,
                         packed ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
     };
-    CR_TRY(op_map(&ta, A, M, Cfg::BM, Cfg::A4));
-    CR_TRY(op_map(&tb, B, N, Cfg::BN, Cfg::B4));
-    CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, Cfg::CHUNK, CU_TENSOR_MAP_SWIZZLE_128B));
-    const int64_t tiles = ((M + Cfg::BM - 1) / Cfg::BM) * ((N + Cfg::BN - 1) / Cfg::BN);
-    const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
+    const int64_t rows_a = Cfg::SWAP ? N : M, rows_b = Cfg::SWAP ? M : N;
+    CR_TRY(op_map(&ta, Cfg::SWAP ? Wc : Xc, rows_a, Cfg::BM, Cfg::A4));
+    CR_TRY(op_map(&tb, Cfg::SWAP ? Xc : Wc, rows_b, Cfg::BN, Cfg::B4));
+    if (Cfg::SWAP) ty = ta;  // stores go straight to Y
+    else CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+    const int64_t units = ((rows_a + Cfg::BM - 1) / Cfg::BM) * ((rows_b + Cfg::BN - 1) / Cfg::BN) * splits;
+    const int grid = static_cast<int>(units < info->sms ? units : info->sms);
     launch_pdl(convrot::gemm_i8_tcgen05_kernel<Cfg>, dim3(grid), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, ta, tb,
-               ty, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sx, sw,
-               static_cast<const __half *>(bias), acc_out);
+               ty, static_cast<int>(rows_a), static_cast<int>(rows_b), static_cast<int>(K), sx, sw,
+               static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out, splits, acc_buf, counters);
     return launch_status("gemm_i8_tcgen05");
 }
 
-// Picks the tile width: the widest tile that still gives every SM work.
-// A4 / B4: activation / weight operand packed int4.
-template <bool A4, bool B4>
-convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *A, const void *B, int64_t M, int64_t N,
+// X4 / W4: activation / weight codes packed int4.
+template <bool X4, bool W4>
+convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const void *Wc, int64_t M, int64_t N,
                              int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
-                             int32_t *acc_out, cudaStream_t st) {
-    const int64_t tiles_m = (M + 127) / 128;
-    const int64_t tiles_256 = tiles_m * ((N + 255) / 256);
-    if (N >= 256 && tiles_256 >= info->sms)
-        return launch_gemm_cfg<convrot::GemmCfg<256, A4, B4>>(info, dev, A, B, M, N, K, sx, sw, bias, Y, acc_out,
-                                                              st);
-    return launch_gemm_cfg<convrot::GemmCfg<128, A4, B4>>(info, dev, A, B, M, N, K, sx, sw, bias, Y, acc_out, st);
+                             int32_t *acc_out, cudaStream_t st, const GemmPlan &p, int32_t *acc_buf = nullptr,
+                             unsigned int *counters = nullptr) {
+    using convrot::GemmCfg;
+    if (p.swap) {
+        if (p.bn == 32)
+            return launch_gemm_cfg<GemmCfg<32, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st,
+                                                              p.splits, acc_buf, counters);
+        if (p.bn == 128)
+            return launch_gemm_cfg<GemmCfg<128, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out,
+                                                               st, p.splits, acc_buf, counters);
+        return launch_gemm_cfg<GemmCfg<256, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st,
+                                                           p.splits, acc_buf, counters);
+    }
+    if (p.bn == 256)
+        return launch_gemm_cfg<GemmCfg<256, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
+                                                     nullptr, nullptr);
+    return launch_gemm_cfg<GemmCfg<128, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1, nullptr,
+                                                 nullptr);
 }
 
 convrot_status_t check_gemm_args(const void *Xq, const float *xs, int64_t M, const void *Wq, const float *ws,
@@ -359,6 +419,20 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits) {
     return round256(codes) + round256(static_cast<size_t>(M) * 4);
 }
 
+size_t convrot_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits) {
+    const size_t base = convrot_workspace_bytes(M, K, bits);
+    if (base == 0 || N < 0) return 0;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
+    } else {
+        cudaGetLastError();
+    }
+    if (M == 0 || N == 0 || K % 128 != 0 || K < 128) return base + kCounterBytes;
+    return base + kCounterBytes + split_buffer_bytes(plan_gemm(sms, M, N, K, true), M, N);
+}
+
 convrot_status_t convrot_quantize_weight(const void *W, int w_dtype, int64_t N, int64_t K, int block, int bits,
                                          int clip_mode, void *Wq, float *w_scale, void *stream) {
     g_last_error.clear();
@@ -406,12 +480,18 @@ convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, i
                                  info->sms, dev);
 }
 
-// Workspace layout of the linears: activation codes (one byte each) then, at
-// the next 256-byte boundary, the per-token scales.
-static void workspace_parts(void *workspace, int64_t M, int64_t K, void **xq, float **xs) {
+// Workspace layout of the linears: activation codes (one byte each); at the
+// next 256-byte boundary the per-token scales; then (when the workspace is
+// large enough) kMaxSplitTiles split-K counters and the int32 M x N sum
+// buffer of a split feature-major GEMM.
+static void workspace_parts(void *workspace, int64_t M, int64_t K, void **xq, float **xs,
+                            unsigned int **counters = nullptr, int32_t **acc_buf = nullptr) {
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     *xq = ws;
     *xs = reinterpret_cast<float *>(ws + round256(static_cast<size_t>(M) * K));
+    uint8_t *extra = ws + round256(static_cast<size_t>(M) * K) + round256(static_cast<size_t>(M) * 4);
+    if (counters) *counters = reinterpret_cast<unsigned int *>(extra);
+    if (acc_buf) *acc_buf = reinterpret_cast<int32_t *>(extra + kCounterBytes);
 }
 
 static convrot_status_t check_linear_shape(int64_t M, int64_t K, int block, int bits, int64_t N) {
@@ -431,8 +511,11 @@ static convrot_status_t check_workspace(const void *workspace, size_t workspace_
     return ok();
 }
 
+// n_features >= 0: the GEMM half's N is known, so exactly the split-K state it
+// will use is zeroed; otherwise everything after the codes and scales, up to
+// the largest split buffer a GEMM over M tokens can use.
 static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, void *workspace,
-                                        size_t workspace_bytes, cudaStream_t st) {
+                                        size_t workspace_bytes, cudaStream_t st, int64_t n_features = -1) {
     CR_REQUIRE(X != nullptr, CONVROT_ERR_INVALID_ARG, "null pointer argument");
     CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
     CR_TRY(check_workspace(workspace, workspace_bytes, M, K, bits));
@@ -441,8 +524,25 @@ static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int
     CR_TRY(current_device(&dev, &info));
     void *xq;
     float *xs;
-    workspace_parts(workspace, M, K, &xq, &xs);
-    return rotate_quant_act_impl(X, M, K, block, bits, false, xq, xs, st, info->sms, dev);
+    unsigned int *counters;
+    workspace_parts(workspace, M, K, &xq, &xs, &counters);
+    // the split-K counters and sum buffer that follow the codes and scales are
+    // zeroed here for the GEMM half
+    const size_t base = convrot_workspace_bytes(M, K, bits);
+    size_t zero_bytes = 0;
+    if (workspace_bytes > base) {
+        size_t cap;
+        if (n_features >= 0) {
+            const GemmPlan p = plan_gemm(info->sms, M, n_features, K, true);
+            cap = kCounterBytes + split_buffer_bytes(p, M, n_features);
+        } else {
+            cap = kCounterBytes + (M <= kSwapMaxTokens ? round256(static_cast<size_t>(M) * kMaxSplitFeatures * 4) : 0);
+        }
+        zero_bytes = (workspace_bytes - base < cap ? workspace_bytes - base : cap) & ~size_t(15);
+    }
+    return rotate_quant_act_impl(X, M, K, block, bits, false, xq, xs, st, info->sms, dev,
+                                 zero_bytes ? reinterpret_cast<uint4 *>(counters) : nullptr,
+                                 static_cast<int64_t>(zero_bytes / 16));
 }
 
 static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace_bytes, int64_t M, int64_t K,
@@ -451,13 +551,23 @@ static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace
     CR_TRY(check_workspace(workspace, workspace_bytes, M, K, bits));
     void *xq;
     float *xs;
-    workspace_parts(const_cast<void *>(workspace), M, K, &xq, &xs);
+    unsigned int *counters;
+    int32_t *acc_buf;
+    workspace_parts(const_cast<void *>(workspace), M, K, &xq, &xs, &counters, &acc_buf);
     CR_TRY(check_gemm_args(xq, xs, M, Wq, w_scale, N, K, bias, Y));
     int dev;
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
-    if (bits == 8) return launch_gemm<false, false>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
-    return launch_gemm<false, true>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st);
+    // split K only when the workspace holds the counters and the sum buffer
+    // (which the activation half zeroed)
+    GemmPlan p = plan_gemm(info->sms, M, N, K, true);
+    const size_t base = convrot_workspace_bytes(M, K, bits) + kCounterBytes;
+    if (p.splits > 1 && workspace_bytes < base + split_buffer_bytes(p, M, N)) p.splits = 1;
+    if (bits == 8)
+        return launch_gemm<false, false>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st, p, acc_buf,
+                                         counters);
+    return launch_gemm<false, true>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st, p, acc_buf,
+                                    counters);
 }
 
 static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t K, const void *Wq,
@@ -468,7 +578,7 @@ static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t 
     if (M == 0 || N == 0) return ok();
     CR_REQUIRE(X && Wq && w_scale && Y, CONVROT_ERR_INVALID_ARG, "null pointer argument");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    CR_TRY(linear_act_impl(X, M, K, block, bits, workspace, workspace_bytes, st));
+    CR_TRY(linear_act_impl(X, M, K, block, bits, workspace, workspace_bytes, st, N));
     return linear_gemm_impl(workspace, workspace_bytes, M, K, bits, Wq, w_scale, N, bias, Y, st);
 }
 
@@ -514,8 +624,9 @@ static convrot_status_t gemm_impl(bool w4, const void *Xq, const float *x_scale,
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (w4) return launch_gemm<true, true>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st);
-    return launch_gemm<false, false>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st);
+    const GemmPlan p = plan_gemm(info->sms, M, N, K, false);  // no workspace: no split-K
+    if (w4) return launch_gemm<true, true>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st, p);
+    return launch_gemm<false, false>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st, p);
 }
 
 convrot_status_t convrot_gemm_w8a8(const int8_t *Xq, const float *x_scale, int64_t M, const int8_t *Wq,

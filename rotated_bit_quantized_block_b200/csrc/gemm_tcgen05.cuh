@@ -7,65 +7,89 @@
 // Method: civarchive.com "SAM 3.1 Multiplex ConvRot" release, "Quantization
 // recipe" (W8A8 / W4A4 operations, per-row scales; INT4 multiplication falls
 // back to INT8 multiplication where the hardware has no INT4 path -- sm_100
-// tcgen05 has no integer-4 kind, so W4A4 tiles are widened to int8 in shared
+// tcgen05 has no integer-4 kind, so int4 tiles are widened to int8 in shared
 // memory before the int8 MMA).
 //
-// Structure: persistent, warp-specialized CTAs (one per SM), output tile
+// Structure: persistent, warp-specialized CTAs (one per SM), accumulator tile
 // 128 x BN, K step 128 bytes.
 //   warp 0      TMA producer (one elected lane): A and B tiles -> smem ring
 //   warp 1      TMEM allocator + MMA issuer (one lane): 4 x tcgen05.mma per K step
-//   warps 2-9   epilogue: tcgen05.ld of the accumulator, scale, fp16, staged
-//               in shared memory and written by TMA bulk stores
-//   warps 10-13 (W4A4 only) nibble -> byte converters between a packed ring
-//               and the MMA ring
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator, scale, fp16, store
+//   warps 10-13 (int4 operands only) nibble -> byte converters between a
+//               packed ring and the MMA ring
 // Two TMEM accumulators (2 x BN columns) let the epilogue of one tile overlap
 // the main loop of the next.  No TMA multicast is used anywhere.
+//
+// Two operand orders:
+//   * token-major (SWAP = false): A = activation codes (128 tokens per tile),
+//     B = weight codes (BN output features); the epilogue stages 32 x 64 fp16
+//     boxes in shared memory and writes them with TMA stores.
+//   * feature-major (SWAP = true, few tokens): A = weight codes (128 output
+//     features per tile), B = activation codes (BN = 32 / 128 / 256 tokens), so
+//     the tensor core is not spent on empty token rows and the weights stream
+//     through a deep ring.  Each epilogue thread owns one output feature and
+//     writes token columns with coalesced stores.  The K loop may be split
+//     across CTAs: every slice adds its int32 partial into a zeroed M x N
+//     buffer (red.add), and the slice that counts in last dequantizes the sum
+//     and zeroes the buffer again.
 #pragma once
 
 #include "device_utils.cuh"
 
 namespace convrot {
 
-// A4 / B4: the activation / weight operand arrives as packed int4 (two codes
-// per byte) and is widened in shared memory; otherwise it is int8 loaded by TMA
-// straight into the MMA ring.  Widened bytes hold 16 * code, so the
-// accumulator carries a factor 16 per widened operand (ACC_SHIFT undoes it).
-template <int BN_, bool A4_, bool B4_>
+// A4 / B4: the MMA's A / B operand arrives as packed int4 (two codes per byte)
+// and is widened in shared memory; otherwise it is int8 loaded by TMA straight
+// into the MMA ring.  Widened bytes hold 16 * code, so the accumulator carries
+// a factor 16 per widened operand (ACC_SHIFT undoes it).
+template <int BN_, bool A4_, bool B4_, bool SWAP_ = false>
 struct GemmCfg {
     static constexpr int BM = 128;
     static constexpr int BN = BN_;
     static constexpr int BK = 128;  // K elements per stage (= bytes of one int8 row segment)
     static constexpr bool A4 = A4_;
     static constexpr bool B4 = B4_;
-    static constexpr bool W4 = A4 || B4;  // some operand is widened by converter warps
+    static constexpr bool SWAP = SWAP_;
+    static constexpr bool W4 = A4 || B4;          // some operand is widened by converter warps
+    static constexpr bool TMA_RING = !(A4 && B4);  // some operand goes straight into the MMA ring
     static constexpr int ACC_SHIFT = (A4 ? 4 : 0) + (B4 ? 4 : 0);
     static constexpr int A_BYTES = BM * BK;
     static constexpr int B_BYTES = BN * BK;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    // MMA ring depth and packed ring depth
-    static constexpr int STAGES = !W4 ? (BN == 256 ? 4 : 6) : A4 ? (BN == 256 ? 2 : 3) : (BN == 256 ? 3 : 4);
-    static constexpr int PSTAGES = !W4 ? 0 : (BN == 256 ? 3 : 4);
     static constexpr int PA_BYTES = A4 ? A_BYTES / 2 : 0;
-    static constexpr int PB_BYTES = B_BYTES / 2;
+    static constexpr int PB_BYTES = B4 ? B_BYTES / 2 : 0;
     static constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
-    static constexpr int CONV_ROWS = (A4 ? BM : 0) + BN;  // rows widened per stage
-    // arrivals completing an MMA stage: the producer (A bytes by TMA) and/or the converters
-    static constexpr int FULL_COUNT = !W4 ? 1 : (A4 ? 128 : 129);
+    static constexpr int PSTAGES = !W4 ? 0 : (!SWAP && BN == 256 ? 3 : 4);
+    static constexpr int CONV_ROWS = (A4 ? BM : 0) + (B4 ? BN : 0);  // rows widened per stage
+    // arrivals completing an MMA stage: the producer (TMA bytes) and/or the 128 converter threads
+    static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + (W4 ? 128 : 0);
     static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int EPI_WARPS = 8;           // two per TMEM lane quarter, each half of the columns
-    static constexpr int EPI_COLS = BN / 2;       // columns per epilogue warp
-    static constexpr int CHUNK = 64;              // columns per output box (two 32-column TMEM loads)
-    static constexpr int OUT_BOX_BYTES = 32 * CHUNK * 2;  // 32 rows x 64 fp16, 128-byte rows
-    static constexpr int OUT_BYTES = EPI_WARPS * OUT_BOX_BYTES;  // one box per epilogue warp
-    static constexpr int SCALE_BYTES = BN * 4 + BN * 2;        // the tile's w_scale (fp32) and bias (fp16)
+    static constexpr int EPI_WARPS = 8;      // two per TMEM lane quarter, each half of the columns
+    static constexpr int EPI_COLS = BN / 2;  // accumulator columns per epilogue warp
+    // token-major: 64-column output boxes (two 32-column TMEM loads);
+    // feature-major: 16- or 32-column TMEM loads, stored directly
+    static constexpr int CHUNK = !SWAP ? 64 : (EPI_COLS < 32 ? EPI_COLS : 32);
+    static constexpr int OUT_BOX_BYTES = 32 * 64 * 2;  // 32 rows x 64 fp16, 128-byte rows
+    static constexpr int OUT_BYTES = SWAP ? 0 : EPI_WARPS * OUT_BOX_BYTES;
+    static constexpr int SCALE_BYTES = BN * 4 + BN * 2;  // the tile's column scale (fp32) and bias (fp16)
     static constexpr int FIRST_CONV_WARP = 2 + EPI_WARPS;
     static constexpr int NUM_THREADS = 32 * (FIRST_CONV_WARP + (W4 ? 4 : 0));
-    static constexpr int NUM_BARRIERS = 2 * STAGES + 2 * PSTAGES + 4 + 1 + 2;
+    static constexpr int FIXED_BARRIERS = 2 * PSTAGES + 4 + 1 + 2 + 2;
+    // MMA ring depth: as many stages as fit in the shared-memory budget (at most 12)
+    static constexpr int SMEM_LIMIT = 232448;
+    static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - PSTAGES * PSTAGE_BYTES - OUT_BYTES - SCALE_BYTES -
+                                       FIXED_BARRIERS * 8 - 16) /
+                                      (STAGE_BYTES + 16);
+    static constexpr int STAGES = STAGES_FIT < 12 ? STAGES_FIT : 12;
+    static constexpr int NUM_BARRIERS = 2 * STAGES + FIXED_BARRIERS;
     static constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * STAGE_BYTES + PSTAGES * PSTAGE_BYTES +
                                       OUT_BYTES + SCALE_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t IDESC = idesc_i8(BM, BN);
-    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
+    static_assert(STAGES >= 2, "pipeline depth");
+    static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+    static_assert(SWAP ? (BN == 32 || BN == 64 || BN == 128 || BN == 256) : (BN % 64 == 0 && BN >= 64 && BN <= 256),
+                  "tile width");
+    static_assert(EPI_COLS % CHUNK == 0, "epilogue chunking");
 };
 
 // Bounded wait used while draining: ignores the abort flag, still time-limited.
@@ -84,9 +108,14 @@ __device__ __forceinline__ uint4 widen_int4x16(uint2 p) {
                       __byte_perm(lo1, hi1, 0x7362));
 }
 
-// Dequantizes 8 accumulators of one row: fp16(fma(fp32(float(acc) * sx), sw[c], bias[c]))
-// (the final multiply-add is one explicit fused operation, so it rounds once).
-// sw_s / bias_s point at the tile's scales staged in shared memory.
+// Dequantizes one accumulator: fp16(fma(fp32(float(acc) * sx), sw, bias)) (the
+// final multiply-add is one explicit fused operation, so it rounds once).
+__device__ __forceinline__ __half dequant1(int32_t a, float sxm, float swn, float bn) {
+    return __float2half_rn(__fmaf_rn(__fmul_rn(__int2float_rn(a), sxm), swn, bn));
+}
+
+// Dequantizes 8 accumulators of one row (token-major order).  sw_s / bias_s
+// point at the tile's scales staged in shared memory.
 template <int SHIFT>
 __device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const float *sw_s, const __half *bias_s,
                                           int32_t *acc_vals) {
@@ -112,20 +141,32 @@ __device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const fl
     return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+// Loads CHUNK (16 or 32) accumulator columns of this warp's 32 TMEM lanes.
+template <int CHUNK>
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[CHUNK]) {
+    if constexpr (CHUNK == 32) tmem_ld_32x32(taddr, r);
+    else tmem_ld_32x16(taddr, r);
+}
+
+// Kernel arguments, in the MMA's terms: the accumulator is M x N (rows of A x
+// rows of B).  Token-major: M = tokens, N = output features.  Feature-major:
+// M = output features, N = tokens.  sx is always the per-token scale, sw the
+// per-feature scale, bias per feature; Y and acc_out are tokens x features.
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmY, int M, int N, int K, const float *__restrict__ sx,
-                           const float *__restrict__ sw, const __half *__restrict__ bias,
-                           int32_t *__restrict__ acc_out) {
+                           const float *__restrict__ sw, const __half *__restrict__ bias, __half *__restrict__ Y,
+                           int32_t *__restrict__ acc_out, int splits, int32_t *__restrict__ acc_buf,
+                           unsigned int *__restrict__ counters) {
     constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, PSTAGES = Cfg::PSTAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ring = smem;                                          // STAGES x (A | B), int8, 128B-swizzled
     uint8_t *pring = ring + STAGES * Cfg::STAGE_BYTES;             // PSTAGES x (A4 | B4), packed, dense rows
     uint8_t *outbuf = pring + PSTAGES * Cfg::PSTAGE_BYTES;         // per epilogue warp: 32 x 64 fp16 box
-    float *sw_s = reinterpret_cast<float *>(outbuf + Cfg::OUT_BYTES);          // [BN] tile w_scale
-    __half *bias_s = reinterpret_cast<__half *>(sw_s + BN);                     // [BN] tile bias
+    float *col_s = reinterpret_cast<float *>(outbuf + Cfg::OUT_BYTES);         // [BN] tile column scale
+    __half *bias_s = reinterpret_cast<__half *>(col_s + BN);                    // [BN] tile bias (token-major)
     uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + Cfg::OUT_BYTES + Cfg::SCALE_BYTES);
     uint64_t *full = bars;                                         // MMA ring: operands ready
     uint64_t *empty = full + STAGES;                               // MMA ring: slot consumed
@@ -136,13 +177,21 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     uint64_t *drain = tmem_empty + 2;                              // MMA completion at exit
     uint64_t *scale_ready = drain + 1;                             // tile scales staged in smem
     uint64_t *scale_free = scale_ready + 1;                        // tile scales no longer read
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(scale_free + 1);
+    uint64_t *partial_done = scale_free + 1;                       // split K: this slice's partial added
+    uint64_t *decided = partial_done + 1;                          // split K: last-slice decision made
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(decided + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *s_last = reinterpret_cast<volatile int *>(tmem_slot + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
     const int num_tiles = tiles_m * tiles_n;
     const int num_kb = K / Cfg::BK;
+    // split K (feature-major only): work unit u is K slice (u % splits) of tile (u / splits)
+    const int num_units = num_tiles * splits;
+    auto unit_tile = [&](int u) { return u / splits; };
+    auto unit_kb0 = [&](int u) { return (u - (u / splits) * splits) * num_kb / splits; };
+    auto unit_kb1 = [&](int u) { return (u - (u / splits) * splits + 1) * num_kb / splits; };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -160,13 +209,15 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         mbar_init(drain, 1);
         mbar_init(scale_ready, 32 * Cfg::EPI_WARPS);
         mbar_init(scale_free, 32 * Cfg::EPI_WARPS);
+        mbar_init(partial_done, 32 * Cfg::EPI_WARPS);
+        mbar_init(decided, 1);
         *abort = 0;
         fence_mbarrier_init();
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
-        tma_prefetch_desc(&tmY);
+        if (!Cfg::SWAP) tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -176,7 +227,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
-    pdl_wait();  // the codes and scales may come from the previous kernel
+    pdl_wait();  // the codes, scales and split-K buffers may come from the previous kernel
     pdl_launch_dependents();
 
     if (warp == 0) {
@@ -192,18 +243,18 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             for (int i = 0; i < STAGES; ++i) filled[i] = false;
             for (int i = 0; i < PSTAGES; ++i) pfilled[i] = false;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            for (int unit = blockIdx.x; ok && unit < num_units; unit += gridDim.x) {
+                const int tile = unit_tile(unit);
                 const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!Cfg::A4) {
+                for (int kb = unit_kb0(unit); kb < unit_kb1(unit); ++kb) {
+                    if (Cfg::TMA_RING) {
                         if (!mbar_wait(&empty[s], ph ^ 1, abort)) {
                             ok = false;
                             break;
                         }
                         uint8_t *dst = ring + s * Cfg::STAGE_BYTES;
-                        const uint32_t bytes = Cfg::B4 ? Cfg::A_BYTES : Cfg::STAGE_BYTES;
-                        mbar_arrive_expect_tx(&full[s], bytes);
-                        tma_load_2d(dst, &tmA, &full[s], kb * Cfg::BK, tm * BM);
+                        mbar_arrive_expect_tx(&full[s], (Cfg::A4 ? 0 : Cfg::A_BYTES) + (Cfg::B4 ? 0 : Cfg::B_BYTES));
+                        if (!Cfg::A4) tma_load_2d(dst, &tmA, &full[s], kb * Cfg::BK, tm * BM);
                         if (!Cfg::B4) tma_load_2d(dst + Cfg::A_BYTES, &tmB, &full[s], kb * Cfg::BK, tn * BN);
                         filled[s] = true;
                         last_parity[s] = ph;
@@ -220,7 +271,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                         uint8_t *dst = pring + ps * Cfg::PSTAGE_BYTES;
                         mbar_arrive_expect_tx(&pfull[ps], Cfg::PSTAGE_BYTES);
                         if (Cfg::A4) tma_load_2d(dst, &tmA, &pfull[ps], kb * (Cfg::BK / 2), tm * BM);
-                        tma_load_2d(dst + Cfg::PA_BYTES, &tmB, &pfull[ps], kb * (Cfg::BK / 2), tn * BN);
+                        if (Cfg::B4) tma_load_2d(dst + Cfg::PA_BYTES, &tmB, &pfull[ps], kb * (Cfg::BK / 2), tn * BN);
                         pfilled[ps] = true;
                         plast_parity[ps] = pph;
                         if (++ps == PSTAGES) {
@@ -231,7 +282,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                 }
             }
             // no bulk copy may still be writing shared memory when the CTA exits
-            // (an MMA stage also waits for its converters when B is widened)
+            // (an MMA stage also waits for its converters when an operand is widened)
             for (int i = 0; i < STAGES; ++i)
                 if (filled[i]) mbar_wait_drain(&full[i], last_parity[i]);
             for (int i = 0; i < PSTAGES; ++i)
@@ -244,13 +295,14 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             uint32_t ph = 0;
             bool ok = true;
             int local = 0;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++local) {
+            for (int unit = blockIdx.x; ok && unit < num_units; unit += gridDim.x, ++local) {
                 const int acc = local & 1;
                 const uint32_t acc_ph = (local >> 1) & 1;
                 if (!mbar_wait(&tmem_empty[acc], acc_ph ^ 1, abort)) break;
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * BN;
-                for (int kb = 0; kb < num_kb; ++kb) {
+                const int kb0 = unit_kb0(unit);
+                for (int kb = kb0; kb < unit_kb1(unit); ++kb) {
                     if (!mbar_wait(&full[s], ph, abort)) {
                         ok = false;
                         break;
@@ -261,7 +313,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < Cfg::BK / 32; ++kk) {
                         umma_i8(d_tmem, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
-                                Cfg::IDESC, (kb | kk) != 0);
+                                Cfg::IDESC, (kb != kb0) || (kk != 0));
                     }
                     umma_commit(&empty[s]);
                     if (++s == STAGES) {
@@ -278,106 +330,186 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         // ------------------------------------------------------------ epilogue
         // Warp w reads TMEM lanes 32*(w%4) .. +31 (its hardware lane quarter)
         // and columns [half * BN/2, (half+1) * BN/2) of the accumulator.  The
-        // tile's w_scale / bias are prefetched into registers one tile ahead
-        // (one column per thread) and staged in shared memory at tile start.
+        // tile's column scales (and, token-major, the bias) are prefetched into
+        // registers one tile ahead (one column per thread) and staged in
+        // shared memory at tile start.
         const int ew = warp - 2;  // 0..7
         const int q = warp & 3;
         const int half = ew >> 2;
-        uint8_t *box = outbuf + ew * Cfg::OUT_BOX_BYTES;
         const int scol = ew * 32 + lane;  // the tile column this thread stages (valid if < BN)
+        const float *col_scale = Cfg::SWAP ? sx : sw;
         auto load_scales = [&](int t, float &wv, __half &bv) {
             wv = 0.0f;
             bv = __float2half_rn(0.0f);
             if (t < num_tiles && scol < BN) {
                 const int col = (t - (t / tiles_n) * tiles_n) * BN + scol;
                 if (col < N) {
-                    wv = __ldg(sw + col);
-                    if (bias != nullptr) bv = bias[col];
+                    wv = __ldg(col_scale + col);
+                    if (!Cfg::SWAP && bias != nullptr) bv = bias[col];
                 }
             }
         };
         float next_w;
         __half next_b;
-        load_scales(blockIdx.x, next_w, next_b);
+        load_scales(unit_tile(blockIdx.x < num_units ? blockIdx.x : 0), next_w, next_b);
         int local = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+        int n_split_units = 0;  // split units handled so far (parity of the split-K barriers)
+        for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++local) {
+            const int tile = unit_tile(unit);
             const int acc = local & 1;
             const uint32_t acc_ph = (local >> 1) & 1;
             if (!mbar_wait(&tmem_full[acc], acc_ph, abort)) break;
             tc_fence_after_sync();
-            // every epilogue thread is done with the previous tile's scales
+            // every epilogue thread is done with the previous unit's scales
             if (local > 0 && !mbar_wait(scale_free, (local - 1) & 1, abort)) break;
             if (scol < BN) {
-                sw_s[scol] = next_w;
+                col_s[scol] = next_w;
                 bias_s[scol] = next_b;
             }
             mbar_arrive(scale_ready);
             if (!mbar_wait(scale_ready, local & 1, abort)) break;
-            load_scales(tile + gridDim.x, next_w, next_b);
+            load_scales(unit + gridDim.x < num_units ? unit_tile(unit + gridDim.x) : num_tiles, next_w, next_b);
             const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
             const int row0 = tm * BM + q * 32;
             const int row = row0 + lane;
             const bool row_ok = row < M;
-            const float sxm = row_ok ? sx[row] : 0.0f;
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+            constexpr int CH = Cfg::CHUNK;
+            constexpr int NCHUNK = Cfg::EPI_COLS / CH;
+            if constexpr (!Cfg::SWAP) {
+                // ---- token-major: row = token; 32 x 64 boxes through shared memory and TMA
+                uint8_t *box = outbuf + ew * Cfg::OUT_BOX_BYTES;
+                const float sxm = row_ok ? sx[row] : 0.0f;
 #pragma unroll 1
-            for (int c = 0; c < Cfg::EPI_COLS / Cfg::CHUNK; ++c) {
-                const int col_local = half * Cfg::EPI_COLS + c * Cfg::CHUNK;
-                uint32_t r[2][32];
-                __syncwarp();  // tcgen05.ld is warp-collective
-                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + col_local;
-                tmem_ld_32x32(taddr, r[0]);
-                tmem_ld_32x32(taddr + 32, r[1]);
-                tmem_ld_wait();
-                if (c == Cfg::EPI_COLS / Cfg::CHUNK - 1) {
-                    // every TMEM read of this tile by this thread is complete
-                    tc_fence_before_sync();
-                    mbar_arrive(&tmem_empty[acc]);
-                }
-                const int col0 = tn * BN + col_local;
-                if (row0 >= M || col0 >= N) continue;  // whole box outside Y (warp-uniform)
-                // the store issued from this box last time must have read it
-                if (lane == 0) bulk_wait_group_read<0>();
-                __syncwarp();
+                for (int c = 0; c < NCHUNK; ++c) {
+                    const int col_local = half * Cfg::EPI_COLS + c * CH;
+                    uint32_t r[2][32];
+                    __syncwarp();  // tcgen05.ld is warp-collective
+                    tmem_ld_32x32(tbase + col_local, r[0]);
+                    tmem_ld_32x32(tbase + col_local + 32, r[1]);
+                    tmem_ld_wait();
+                    if (c == NCHUNK - 1) {
+                        // every TMEM read of this unit by this thread is complete
+                        tc_fence_before_sync();
+                        mbar_arrive(&tmem_empty[acc]);
+                    }
+                    const int col0 = tn * BN + col_local;
+                    if (row0 >= M || col0 >= N) continue;  // whole box outside Y (warp-uniform)
+                    // the store issued from this box last time must have read it
+                    if (lane == 0) bulk_wait_group_read<0>();
+                    __syncwarp();
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {  // 8 columns per 16-byte chunk
-                    int32_t av[8];
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (row_ok && col0 + 8 * g < N) {
-                        v = dequant8<Cfg::ACC_SHIFT>(r[g >> 2] + 8 * (g & 3), sxm, sw_s + col_local + 8 * g,
-                                              bias_s + col_local + 8 * g, av);
-                        if (acc_out != nullptr) {
-                            int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0 + 8 * g);
-                            dst[0] = make_int4(av[0], av[1], av[2], av[3]);
-                            dst[1] = make_int4(av[4], av[5], av[6], av[7]);
+                    for (int g = 0; g < 8; ++g) {  // 8 columns per 16-byte chunk
+                        int32_t av[8];
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (row_ok && col0 + 8 * g < N) {
+                            v = dequant8<Cfg::ACC_SHIFT>(r[g >> 2] + 8 * (g & 3), sxm, col_s + col_local + 8 * g,
+                                                         bias_s + col_local + 8 * g, av);
+                            if (acc_out != nullptr) {
+                                int4 *dst =
+                                    reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0 + 8 * g);
+                                dst[0] = make_int4(av[0], av[1], av[2], av[3]);
+                                dst[1] = make_int4(av[4], av[5], av[6], av[7]);
+                            }
+                        }
+                        // 128-byte rows, 16-byte chunk g stored at g ^ (row & 7) (128B swizzle)
+                        *reinterpret_cast<uint4 *>(box + lane * 128 + ((g ^ (lane & 7)) << 4)) = v;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmY, box, col0, row0);
+                        bulk_commit_group();
+                    }
+                }
+            } else {
+                // ---- feature-major: row = output feature f, columns = tokens
+                const int f = row;
+                const float swf = row_ok ? sw[f] : 0.0f;
+                const float bf = (row_ok && bias != nullptr) ? __half2float(bias[f]) : 0.0f;
+                const int tok_base = tn * BN + half * Cfg::EPI_COLS;
+#pragma unroll 1
+                for (int c = 0; c < NCHUNK; ++c) {
+                    uint32_t r[CH];
+                    __syncwarp();
+                    tmem_ld_chunk<CH>(tbase + half * Cfg::EPI_COLS + c * CH, r);
+                    tmem_ld_wait();
+                    if (c == NCHUNK - 1) {
+                        tc_fence_before_sync();
+                        mbar_arrive(&tmem_empty[acc]);
+                    }
+                    if (!row_ok) continue;
+#pragma unroll
+                    for (int j = 0; j < CH; ++j) {
+                        const int tok = tok_base + c * CH + j;
+                        if (tok >= N) break;
+                        const int64_t o = static_cast<int64_t>(tok) * M + f;
+                        if (splits > 1) {
+                            atomicAdd(acc_buf + o, static_cast<int32_t>(r[j]));  // result unused: a reduction
+                        } else {
+                            const int32_t a = static_cast<int32_t>(r[j]) >> Cfg::ACC_SHIFT;
+                            Y[o] = dequant1(a, col_s[half * Cfg::EPI_COLS + c * CH + j], swf, bf);
+                            if (acc_out != nullptr) acc_out[o] = a;
                         }
                     }
-                    // 128-byte rows, 16-byte chunk g stored at g ^ (row & 7) (128B swizzle)
-                    *reinterpret_cast<uint4 *>(box + lane * 128 + ((g ^ (lane & 7)) << 4)) = v;
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmY, box, col0, row0);
-                    bulk_commit_group();
+                if (splits > 1) {
+                    __threadfence();  // this slice's additions are visible device-wide before it is counted
+                    mbar_arrive(partial_done);
+                    if (ew == 0 && lane == 0) {
+                        int last = 0;
+                        if (mbar_wait(partial_done, n_split_units & 1, abort)) {
+                            __threadfence();
+                            const unsigned int before = atomicAdd(&counters[tile], 1u);
+                            last = before == static_cast<unsigned int>(splits - 1);
+                            if (last) counters[tile] = 0u;  // ready for the next call
+                            __threadfence();               // the sum is read after the count
+                        }
+                        *s_last = last;
+                        mbar_arrive(decided);
+                    }
+                    if (!mbar_wait(decided, n_split_units & 1, abort)) break;
+                    ++n_split_units;
+                    if (*s_last != 0 && row_ok) {
+#pragma unroll 1
+                        for (int c = 0; c < NCHUNK; ++c) {
+                            int32_t v[CH];
+#pragma unroll
+                            for (int j = 0; j < CH; ++j) {
+                                const int tok = tok_base + c * CH + j;
+                                v[j] = tok < N ? __ldcg(acc_buf + static_cast<int64_t>(tok) * M + f) : 0;
+                            }
+#pragma unroll
+                            for (int j = 0; j < CH; ++j) {
+                                const int tok = tok_base + c * CH + j;
+                                if (tok >= N) break;
+                                const int64_t o = static_cast<int64_t>(tok) * M + f;
+                                acc_buf[o] = 0;  // zero again for the next call
+                                const int32_t a = v[j] >> Cfg::ACC_SHIFT;
+                                Y[o] = dequant1(a, col_s[half * Cfg::EPI_COLS + c * CH + j], swf, bf);
+                                if (acc_out != nullptr) acc_out[o] = a;
+                            }
+                        }
+                    }
                 }
             }
             mbar_arrive(scale_free);
         }
-        if (lane == 0) bulk_wait_group_all();
+        if (!Cfg::SWAP && lane == 0) bulk_wait_group_all();
     } else if (Cfg::W4) {
         // ------------------------------------------------------------ int4 -> int8 converters
         const int ct = threadIdx.x - 32 * Cfg::FIRST_CONV_WARP;  // 0..127
         int ps = 0, us = 0;
         uint32_t pph = 0, uph = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-            for (int kb = 0; kb < num_kb; ++kb) {
+        for (int unit = blockIdx.x; ok && unit < num_units; unit += gridDim.x) {
+            for (int kb = unit_kb0(unit); kb < unit_kb1(unit); ++kb) {
                 if (!mbar_wait(&pfull[ps], pph, abort) || !mbar_wait(&empty[us], uph ^ 1, abort)) {
                     ok = false;
                     break;
                 }
                 const uint8_t *src = pring + ps * Cfg::PSTAGE_BYTES;
-                // widened rows: A (if packed) then B, in the MMA ring's layout
+                // widened rows (A if packed, then B if packed) in the MMA ring's layout
                 uint8_t *dst = ring + us * Cfg::STAGE_BYTES + (Cfg::A4 ? 0 : Cfg::A_BYTES);
                 constexpr int PIECES = Cfg::CONV_ROWS * (Cfg::BK / 16);  // 16 codes per piece
 #pragma unroll 4

@@ -244,7 +244,9 @@ __host__ __device__ constexpr int act_smem_bytes(int threads) { return (threads 
 template <int LOG2B, int BITS, bool PACKED>
 __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__restrict__ X, int64_t M, int K,
                                                                 int rows, void *__restrict__ Xq,
-                                                                float *__restrict__ x_scale) {
+                                                                float *__restrict__ x_scale,
+                                                                uint4 *__restrict__ zero16,
+                                                                int64_t n_zero16) {
     extern __shared__ __align__(16) uint8_t act_smem[];
     __shared__ unsigned int s_amax[kMaxRowsPerCta];
     __shared__ float s_fac[kMaxRowsPerCta];
@@ -271,6 +273,10 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
 #pragma unroll
         for (int j = 0; j < 4; ++j) raw[j] = make_uint4(0, 0, 0, 0);
     }
+    // (while the row loads are in flight) the linear's split-K counters and sum buffer start at zero for the GEMM that follows
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + tid; i < n_zero16;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        zero16[i] = make_uint4(0u, 0u, 0u, 0u);
     if (tid < rows) s_amax[tid] = 0u;
     float2 a[4][4];
 #pragma unroll

@@ -110,3 +110,16 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         binding.convrot_rotate_quant_act(torch.zeros(4, 128, dtype=torch.float16), 64, 8)
+
+
+def test_linear_workspace_bytes_adds_split_k_room(lib):
+    ws, lws = lib.convrot_workspace_bytes, lib.convrot_linear_workspace_bytes
+    for bits in (8, 4):
+        for M, K, N in [(1, 4096, 4096), (16, 1024, 3072), (5184, 4096, 1024), (16384, 4096, 4096)]:
+            assert lws(M, K, N, bits) >= ws(M, K, bits) + 2048
+    # a single row against a 4096 x 4096 weight has too few tiles: room for partials
+    assert lws(1, 4096, 4096, 8) > ws(1, 4096, 8) + 2048
+    # thousands of output tiles: no split, only the counters
+    assert lws(16384, 4096, 4096, 8) == ws(16384, 4096, 8) + 2048
+    assert lws(-1, 4096, 4096, 8) == 0
+    assert lws(4, 4096, 4096, 5) == 0

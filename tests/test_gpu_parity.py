@@ -308,3 +308,38 @@ def test_linear_two_stage_entry_points_equal_the_linear(bits):
     cr.convrot_linear_quant_act(Xd, w.block, bits, ws)
     y2 = host(cr.convrot_linear_gemm(ws, 700, W.shape[1], bits, Wq, sw, bias=bd))
     assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
+
+
+SPLIT_CASES = [(1, 4096, 4096), (16, 4096, 4096), (100, 1024, 4096), (700, 1024, 4096), (5184, 1024, 4096)]
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("M,N,K", SPLIT_CASES)
+def test_linear_split_k_bit_exact(M, N, K, bits):
+    """With the larger workspace the linear may split K across CTAs; the int32
+    sum of the slices is exact, so the output equals the unsplit linear's and
+    the oracle's GEMM of the same codes, bit for bit, on every call."""
+    X = wl.activations(M, K, 0.01, 30.0, seed=M + 7)
+    W = wl.weight(N, K, 0.02, seed=N + 7)
+    bias = wl.bias(N, seed=3)
+    Xd, bd = dev(X), dev(bias)
+    Wq, sw = cr.convrot_quantize_weight(dev(W), 128, bits, cr.CLIP_ABSMAX)
+    fn = cr.convrot_linear_w8a8 if bits == 8 else cr.convrot_linear_w4a4
+    small = cr.convrot_workspace_bytes(M, K, bits)
+    big = cr.convrot_linear_workspace_bytes(M, K, N, bits)
+    assert big >= small + 2048
+    ws_small = torch.empty(small, dtype=torch.uint8, device="cuda")
+    ws_big = torch.empty(big, dtype=torch.uint8, device="cuda")
+    y_ref = host(fn(Xd, Wq, sw, 128, bias=bd, workspace=ws_small))
+    outs = [host(fn(Xd, Wq, sw, 128, bias=bd, workspace=ws_big)) for _ in range(3)]
+    for y in outs:
+        assert np.array_equal(y.view(np.uint16), y_ref.view(np.uint16))
+    # the workspace starts with the activation codes (one per byte) and, at the
+    # next 256-byte boundary, the per-token scales
+    raw = host(ws_big)
+    qx = raw[: M * K].view(np.int8).reshape(M, K)
+    off = (M * K + 255) // 256 * 256
+    sx = raw[off: off + 4 * M].view(np.float32)
+    qw = unpack(host(Wq), bits)
+    yr = oracle.gemm_dequant(qx, sx, qw, host(sw), bias)
+    assert np.array_equal(outs[0].view(np.uint16), yr.view(np.uint16))
