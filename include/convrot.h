@@ -111,8 +111,8 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
 
 /*
  * Workspace size that also lets the linear split the K loop of its GEMM across
- * SMs.  For few tokens (M <= 256) the GEMM runs feature-major (128 output
- * features per tile) and has too few tiles to fill the GPU; with this
+ * SMs.  For few tokens (M <= 128) the GEMM runs feature-major (128 output
+ * features x 32 tokens per tile) and has too few tiles to fill the GPU; with this
  * workspace the K slices of a tile run on separate SMs and add their int32
  * partials into an M x N buffer.  Size: convrot_workspace_bytes(M, K, bits)
  * plus 2 KB of split-K counters plus that buffer (rounded up to 256 bytes)
@@ -156,7 +156,7 @@ convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const 
  * separately (same arguments, same workspace layout): first rotate and
  * quantize X into the workspace, then run the integer GEMM + dequant from it.
  * The workspace must not be reused by another linear in between.  Not knowing
- * N, convrot_linear_quant_act zeroes everything after the scales (for M <= 256
+ * N, convrot_linear_quant_act zeroes everything after the scales (for M <= 128
  * at most the split state of a GEMM with N <= 32768; for larger M only the
  * counters).
  */

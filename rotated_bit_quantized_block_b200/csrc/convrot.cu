@@ -274,23 +274,27 @@ struct GemmPlan {
 
 constexpr int kMaxSplitTiles = 512;              // split-K counters in a linear's workspace
 constexpr size_t kCounterBytes = kMaxSplitTiles * 4;
-constexpr int64_t kSwapMaxTokens = 256;          // feature-major below this many tokens
+constexpr int64_t kSwapMaxTokens = 128;          // feature-major up to this many tokens
+constexpr int kSwapTokens = 32;                  // token tile of the feature-major GEMM
 constexpr int64_t kMaxSplitFeatures = 32768;     // split K only for N up to this
 
-// Few tokens: feature-major tiles (128 features x 32 / 128 / 256 tokens), K
-// split so that the tiles x splits units cover the SMs (at most 8 slices, each
-// at least two 128-deep K steps).  Otherwise token-major 128 x 256 tiles,
+// Few tokens: feature-major tiles (128 features x 32 tokens), K split so that
+// the tiles x splits units cover the SMs (at most 8 slices, each at least 8
+// K steps of 128: a split costs a few microseconds of counting and re-reading,
+// which shorter slices do not repay).  Otherwise token-major 128 x 256 tiles,
 // narrowed to 128 when 256-wide tiles would leave more than half the SMs idle.
+// (Measured on B200 with CUDA-graph launches: feature-major wins up to 128
+// tokens, token-major from 192.)
 GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split) {
     GemmPlan p;
     if (M <= kSwapMaxTokens) {
         p.swap = true;
-        p.bn = M <= 32 ? 32 : (M <= 128 ? 128 : 256);
+        p.bn = kSwapTokens;
         p.tiles = ((N + 127) / 128) * ((M + p.bn - 1) / p.bn);
         if (allow_split && p.tiles > 0 && p.tiles <= kMaxSplitTiles && N <= kMaxSplitFeatures) {
             int64_t s = sms / p.tiles;
             if (s > 8) s = 8;
-            if (s > K / 256) s = K / 256;
+            if (s > K / 1024) s = K / 1024;
             if (s >= 2) p.splits = static_cast<int>(s);
         }
         return p;
@@ -353,16 +357,9 @@ convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const vo
                              int32_t *acc_out, cudaStream_t st, const GemmPlan &p, int32_t *acc_buf = nullptr,
                              unsigned int *counters = nullptr) {
     using convrot::GemmCfg;
-    if (p.swap) {
-        if (p.bn == 32)
-            return launch_gemm_cfg<GemmCfg<32, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st,
-                                                              p.splits, acc_buf, counters);
-        if (p.bn == 128)
-            return launch_gemm_cfg<GemmCfg<128, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out,
-                                                               st, p.splits, acc_buf, counters);
-        return launch_gemm_cfg<GemmCfg<256, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st,
-                                                           p.splits, acc_buf, counters);
-    }
+    if (p.swap)
+        return launch_gemm_cfg<GemmCfg<kSwapTokens, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y,
+                                                                   acc_out, st, p.splits, acc_buf, counters);
     if (p.bn == 256)
         return launch_gemm_cfg<GemmCfg<256, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
                                                      nullptr, nullptr);

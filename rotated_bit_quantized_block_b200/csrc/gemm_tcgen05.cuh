@@ -25,7 +25,7 @@
 //     B = weight codes (BN output features); the epilogue stages 32 x 64 fp16
 //     boxes in shared memory and writes them with TMA stores.
 //   * feature-major (SWAP = true, few tokens): A = weight codes (128 output
-//     features per tile), B = activation codes (BN = 32 / 128 / 256 tokens), so
+//     features per tile), B = activation codes (BN tokens, e.g. 32), so
 //     the tensor core is not spent on empty token rows and the weights stream
 //     through a deep ring.  Each epilogue thread owns one output feature and
 //     writes token columns with coalesced stores.  The K loop may be split
