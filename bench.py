@@ -66,6 +66,49 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# ------------------------------------------------------------------------------------------ traffic
+
+CSRC = os.path.join(ROOT, "rotated_bit_quantized_block_b200", "csrc")
+GEMM_SOURCES = ("gemm_tcgen05.cuh", "device_utils.cuh")
+ACT_SOURCES = ("rotate_quant.cuh", "device_utils.cuh")
+
+
+def source_digest(names) -> str:
+    """sha256 (first 16 hex digits) of the kernel sources, in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(CSRC, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload
+    (profiles/<workload>_dram.txt), per kernel and linear; a kernel whose
+    sources changed since the capture gets None."""
+    path = os.path.join(ROOT, "profiles", f"{workload}_dram.txt")
+    out = {"gemm": None, "act": None}
+    if not os.path.exists(path):
+        return out
+    digests, rows = {}, {"gemm": {}, "act": {}}
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if line.endswith(":") or ": " in line:
+                k, v = line.split(":", 1)
+                digests[k.strip()] = v.strip()
+                continue
+            kind, linear, rd, wr = line.split()
+            rows[kind][linear] = int(rd) + int(wr)
+    for kind, names in (("gemm", GEMM_SOURCES), ("act", ACT_SOURCES)):
+        if rows[kind] and digests.get(f"{kind}_source_digest") == source_digest(names):
+            out[kind] = rows[kind]
+    return out
+
+
 # ------------------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -377,9 +420,16 @@ def ours_arm(args, w, rank, world, local_rank):
     int8_peak = 2.0 * peaks["bf16_tflops"]  # dense int8 = 2 x dense bf16 (4.5 vs 2.25 POPS nominal)
     per_linear_ms = [statistics.mean(gemm_ms[s][i] for s in range(args.steps)) for i in range(n_lin)]
     per_linear_act_ms = [statistics.mean(act_ms[s][i] for s in range(args.steps)) for i in range(n_lin)]
+    traffic = load_traffic(w.name)
+    gemm_traffic = traffic["gemm"]
     roofline = {
         "bound": "tensor", "achieved": achieved_tops, "peak": int8_peak, "unit": "TOPS",
-        "frac": achieved_tops / int8_peak, "traffic": None,
+        "frac": achieved_tops / int8_peak,
+        # mean DRAM bytes per GEMM launch of one step, from the committed ncu capture
+        "traffic": (statistics.mean(gemm_traffic.values()) if gemm_traffic else None),
+        "traffic_per_linear": gemm_traffic,
+        "algorithmic_bytes_per_linear": {l.name: w.M * l.K + l.N * l.K * w.bits // 8 + 2 * w.M * l.N + 4 * w.M + 4 * l.N
+                                         for l in w.linears},
         "kernel": "gemm_i8_tcgen05 (int8 x int8 -> int32, fused dequant epilogue)",
         "peak_note": f"dense int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s",
         "timing": "second timed pass of the same steps with CUDA events around every kernel launch",
@@ -390,9 +440,13 @@ def ours_arm(args, w, rank, world, local_rank):
     act_bytes = [w.M * l.K * 2 + w.M * l.K * w.bits // 8 + 4 * w.M for l in w.linears]
     act_total_ms = sum(per_linear_act_ms)
     act_gbs = sum(act_bytes) / (act_total_ms / 1000.0) / 1e9
+    act_traffic = traffic["act"]
     rotate_quant = {
         "bound": "hbm", "achieved": act_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": act_gbs / peaks["hbm_gbs"], "kernel": "act_rotate_quant",
+        "traffic": (statistics.mean(act_traffic.values()) if act_traffic else None),
+        "traffic_per_linear": act_traffic,
+        "algorithmic_bytes_per_linear": {l.name: b for l, b in zip(w.linears, act_bytes)},
         "per_linear_ms": {l.name: round(t, 5) for l, t in zip(w.linears, per_linear_act_ms)},
         "per_linear_gbs": {l.name: round(b / (t / 1000) / 1e9, 1)
                            for l, b, t in zip(w.linears, act_bytes, per_linear_act_ms)},
