@@ -114,27 +114,24 @@ __device__ __forceinline__ __half dequant1(int32_t a, float sxm, float swn, floa
     return __float2half_rn(__fmaf_rn(__fmul_rn(__int2float_rn(a), sxm), swn, bn));
 }
 
-// Dequantizes 8 accumulators of one row (token-major order).  sw_s / bias_s
-// point at the tile's scales staged in shared memory.
+// Dequantizes 8 accumulators of one row (token-major order).  sw_s / b_s
+// point at the tile's scale (fp32) and bias (fp16) staged in shared memory.
 template <int SHIFT>
-__device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const float *sw_s, const __half *bias_s,
-                                          int32_t *acc_vals) {
+__device__ __forceinline__ uint4 dequant8(const uint32_t *r, float sxm, const float *sw_s, const __half *b_s) {
     const float4 w0 = *reinterpret_cast<const float4 *>(sw_s);
     const float4 w1 = *reinterpret_cast<const float4 *>(sw_s + 4);
-    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    const uint4 braw = *reinterpret_cast<const uint4 *>(bias_s);
+    const float2 wv[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w), make_float2(w1.x, w1.y),
+                          make_float2(w1.z, w1.w)};
+    const uint4 braw = *reinterpret_cast<const uint4 *>(b_s);
     const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
     uint32_t out[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int32_t a0 = static_cast<int32_t>(r[2 * i]) >> SHIFT;
         const int32_t a1 = static_cast<int32_t>(r[2 * i + 1]) >> SHIFT;
-        acc_vals[2 * i] = a0;
-        acc_vals[2 * i + 1] = a1;
-        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&bw[i]));
         float2 t = make_float2(__int2float_rn(a0), __int2float_rn(a1));
         t = __fmul2_rn(t, make_float2(sxm, sxm));
-        t = __ffma2_rn(t, make_float2(wv[2 * i], wv[2 * i + 1]), b);
+        t = __ffma2_rn(t, wv[i], __half22float2(*reinterpret_cast<const __half2 *>(&bw[i])));
         const __half2 h = __floats2half2_rn(t.x, t.y);
         out[i] = *reinterpret_cast<const uint32_t *>(&h);
     }
@@ -398,22 +395,35 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     // the store issued from this box last time must have read it
                     if (lane == 0) bulk_wait_group_read<0>();
                     __syncwarp();
+                    // 128-byte rows, 16-byte chunk g stored at g ^ (row & 7) (128B swizzle)
+                    uint8_t *brow = box + lane * 128;
+                    const int xr = (lane & 7) << 4;
+                    const float *sw_c = col_s + col_local;
+                    const __half *b_c = bias_s + col_local;
+                    if (row_ok && col0 + 64 <= N && acc_out == nullptr) {
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) {  // 8 columns per 16-byte chunk
-                        int32_t av[8];
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (row_ok && col0 + 8 * g < N) {
-                            v = dequant8<Cfg::ACC_SHIFT>(r[g >> 2] + 8 * (g & 3), sxm, col_s + col_local + 8 * g,
-                                                         bias_s + col_local + 8 * g, av);
-                            if (acc_out != nullptr) {
-                                int4 *dst =
-                                    reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0 + 8 * g);
-                                dst[0] = make_int4(av[0], av[1], av[2], av[3]);
-                                dst[1] = make_int4(av[4], av[5], av[6], av[7]);
+                        for (int g = 0; g < 8; ++g)
+                            *reinterpret_cast<uint4 *>(brow + ((g << 4) ^ xr)) =
+                                dequant8<Cfg::ACC_SHIFT>(r[g >> 2] + 8 * (g & 3), sxm, sw_c + 8 * g, b_c + 8 * g);
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) {  // 8 columns per 16-byte chunk
+                            uint4 v = make_uint4(0, 0, 0, 0);
+                            if (row_ok && col0 + 8 * g < N) {
+                                const uint32_t *rg = r[g >> 2] + 8 * (g & 3);
+                                v = dequant8<Cfg::ACC_SHIFT>(rg, sxm, sw_c + 8 * g, b_c + 8 * g);
+                                if (acc_out != nullptr) {
+                                    int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N +
+                                                                         col0 + 8 * g);
+                                    constexpr int SH = Cfg::ACC_SHIFT;
+                                    dst[0] = make_int4(static_cast<int32_t>(rg[0]) >> SH, static_cast<int32_t>(rg[1]) >> SH,
+                                                       static_cast<int32_t>(rg[2]) >> SH, static_cast<int32_t>(rg[3]) >> SH);
+                                    dst[1] = make_int4(static_cast<int32_t>(rg[4]) >> SH, static_cast<int32_t>(rg[5]) >> SH,
+                                                       static_cast<int32_t>(rg[6]) >> SH, static_cast<int32_t>(rg[7]) >> SH);
+                                }
                             }
+                            *reinterpret_cast<uint4 *>(brow + ((g << 4) ^ xr)) = v;
                         }
-                        // 128-byte rows, 16-byte chunk g stored at g ^ (row & 7) (128B swizzle)
-                        *reinterpret_cast<uint4 *>(box + lane * 128 + ((g ^ (lane & 7)) << 4)) = v;
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
