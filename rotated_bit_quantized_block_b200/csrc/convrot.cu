@@ -341,7 +341,7 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, cons
     CR_TRY(op_map(&ta, Cfg::SWAP ? Wc : Xc, rows_a, Cfg::BM, Cfg::A4));
     CR_TRY(op_map(&tb, Cfg::SWAP ? Xc : Wc, rows_b, Cfg::BN, Cfg::B4));
     if (Cfg::SWAP) ty = ta;  // stores go straight to Y
-    else CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+    else CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
     const int64_t units = ((rows_a + Cfg::BM - 1) / Cfg::BM) * ((rows_b + Cfg::BN - 1) / Cfg::BN) * splits;
     const int grid = static_cast<int>(units < info->sms ? units : info->sms);
     launch_pdl(convrot::gemm_i8_tcgen05_kernel<Cfg>, dim3(grid), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, ta, tb,

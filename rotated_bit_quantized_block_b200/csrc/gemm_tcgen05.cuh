@@ -14,15 +14,16 @@
 // 128 x BN, K step 128 bytes.
 //   warp 0      TMA producer (one elected lane): A and B tiles -> smem ring
 //   warp 1      TMEM allocator + MMA issuer (one lane): 4 x tcgen05.mma per K step
-//   warps 2-9   epilogue: tcgen05.ld of the accumulator, scale, fp16, store
-//   warps 10-13 (int4 operands only) nibble -> byte converters between a
-//               packed ring and the MMA ring
+//   epilogue    16 warps (token-major) or 8 (feature-major): tcgen05.ld of
+//               the accumulator, scale, fp16, store
+//   converters  4 warps (int4 operands only): nibble -> byte widening between
+//               a packed ring and the MMA ring
 // Two TMEM accumulators (2 x BN columns) let the epilogue of one tile overlap
 // the main loop of the next.  No TMA multicast is used anywhere.
 //
 // Two operand orders:
 //   * token-major (SWAP = false): A = activation codes (128 tokens per tile),
-//     B = weight codes (BN output features); the epilogue stages 32 x 64 fp16
+//     B = weight codes (BN output features); the epilogue stages 32 x 32 fp16
 //     boxes in shared memory and writes them with TMA stores.
 //   * feature-major (SWAP = true, few tokens): A = weight codes (128 output
 //     features per tile), B = activation codes (BN tokens, e.g. 32), so
@@ -64,12 +65,14 @@ struct GemmCfg {
     // arrivals completing an MMA stage: the producer (TMA bytes) and/or the 128 converter threads
     static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + (W4 ? 128 : 0);
     static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int EPI_WARPS = 8;      // two per TMEM lane quarter, each half of the columns
-    static constexpr int EPI_COLS = BN / 2;  // accumulator columns per epilogue warp
-    // token-major: 64-column output boxes (two 32-column TMEM loads);
+    // epilogue warps: per TMEM lane quarter, EPI_WARPS / 4 warps split the columns
+    // (token-major: four, so that enough warps hide the dequant's latencies)
+    static constexpr int EPI_WARPS = SWAP ? 8 : 16;
+    static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // accumulator columns per epilogue warp
+    // token-major: 32-column chunks (one TMEM load, one 32 x 32 fp16 output box);
     // feature-major: 16- or 32-column TMEM loads, stored directly
-    static constexpr int CHUNK = !SWAP ? 64 : (EPI_COLS < 32 ? EPI_COLS : 32);
-    static constexpr int OUT_BOX_BYTES = 32 * 64 * 2;  // 32 rows x 64 fp16, 128-byte rows
+    static constexpr int CHUNK = !SWAP ? 32 : (EPI_COLS < 32 ? EPI_COLS : 32);
+    static constexpr int OUT_BOX_BYTES = 32 * 32 * 2;  // 32 rows x 32 fp16, 64-byte rows
     static constexpr int OUT_BYTES = SWAP ? 0 : EPI_WARPS * OUT_BOX_BYTES;
     static constexpr int SCALE_BYTES = BN * 4 + BN * 2;  // the tile's column scale (fp32) and bias (fp16)
     static constexpr int FIRST_CONV_WARP = 2 + EPI_WARPS;
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ring = smem;                                          // STAGES x (A | B), int8, 128B-swizzled
     uint8_t *pring = ring + STAGES * Cfg::STAGE_BYTES;             // PSTAGES x (A4 | B4), packed, dense rows
-    uint8_t *outbuf = pring + PSTAGES * Cfg::PSTAGE_BYTES;         // per epilogue warp: 32 x 64 fp16 box
+    uint8_t *outbuf = pring + PSTAGES * Cfg::PSTAGE_BYTES;         // per epilogue warp: 32 x 32 fp16 box
     float *col_s = reinterpret_cast<float *>(outbuf + Cfg::OUT_BYTES);         // [BN] tile column scale
     __half *bias_s = reinterpret_cast<__half *>(col_s + BN);                    // [BN] tile bias (token-major)
     uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + Cfg::OUT_BYTES + Cfg::SCALE_BYTES);
@@ -326,13 +329,13 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     } else if (warp < Cfg::FIRST_CONV_WARP) {
         // ------------------------------------------------------------ epilogue
         // Warp w reads TMEM lanes 32*(w%4) .. +31 (its hardware lane quarter)
-        // and columns [half * BN/2, (half+1) * BN/2) of the accumulator.  The
+        // and columns [cg * EPI_COLS, (cg+1) * EPI_COLS) of the accumulator.  The
         // tile's column scales (and, token-major, the bias) are prefetched into
         // registers one tile ahead (one column per thread) and staged in
         // shared memory at tile start.
-        const int ew = warp - 2;  // 0..7
+        const int ew = warp - 2;  // 0 .. EPI_WARPS-1
         const int q = warp & 3;
-        const int half = ew >> 2;
+        const int cg = ew >> 2;   // column group
         const int scol = ew * 32 + lane;  // the tile column this thread stages (valid if < BN)
         const float *col_scale = Cfg::SWAP ? sx : sw;
         auto load_scales = [&](int t, float &wv, __half &bv) {
@@ -374,16 +377,18 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             constexpr int CH = Cfg::CHUNK;
             constexpr int NCHUNK = Cfg::EPI_COLS / CH;
             if constexpr (!Cfg::SWAP) {
-                // ---- token-major: row = token; 32 x 64 boxes through shared memory and TMA
+                // ---- token-major: row = token; 32 x 32 boxes through shared memory and TMA
                 uint8_t *box = outbuf + ew * Cfg::OUT_BOX_BYTES;
                 const float sxm = row_ok ? sx[row] : 0.0f;
+                // 64-byte rows, 16-byte chunk g stored at g ^ ((row / 2) & 3) (64B swizzle)
+                uint8_t *brow = box + lane * 64;
+                const int xr = ((lane >> 1) & 3) << 4;
 #pragma unroll 1
                 for (int c = 0; c < NCHUNK; ++c) {
-                    const int col_local = half * Cfg::EPI_COLS + c * CH;
-                    uint32_t r[2][32];
+                    const int col_local = cg * Cfg::EPI_COLS + c * CH;
+                    uint32_t r[32];
                     __syncwarp();  // tcgen05.ld is warp-collective
-                    tmem_ld_32x32(tbase + col_local, r[0]);
-                    tmem_ld_32x32(tbase + col_local + 32, r[1]);
+                    tmem_ld_32x32(tbase + col_local, r);
                     tmem_ld_wait();
                     if (c == NCHUNK - 1) {
                         // every TMEM read of this unit by this thread is complete
@@ -395,22 +400,19 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     // the store issued from this box last time must have read it
                     if (lane == 0) bulk_wait_group_read<0>();
                     __syncwarp();
-                    // 128-byte rows, 16-byte chunk g stored at g ^ (row & 7) (128B swizzle)
-                    uint8_t *brow = box + lane * 128;
-                    const int xr = (lane & 7) << 4;
                     const float *sw_c = col_s + col_local;
                     const __half *b_c = bias_s + col_local;
-                    if (row_ok && col0 + 64 <= N && acc_out == nullptr) {
+                    if (row_ok && col0 + 32 <= N && acc_out == nullptr) {
 #pragma unroll
-                        for (int g = 0; g < 8; ++g)
+                        for (int g = 0; g < 4; ++g)
                             *reinterpret_cast<uint4 *>(brow + ((g << 4) ^ xr)) =
-                                dequant8<Cfg::ACC_SHIFT>(r[g >> 2] + 8 * (g & 3), sxm, sw_c + 8 * g, b_c + 8 * g);
+                                dequant8<Cfg::ACC_SHIFT>(r + 8 * g, sxm, sw_c + 8 * g, b_c + 8 * g);
                     } else {
 #pragma unroll
-                        for (int g = 0; g < 8; ++g) {  // 8 columns per 16-byte chunk
+                        for (int g = 0; g < 4; ++g) {  // 8 columns per 16-byte chunk
                             uint4 v = make_uint4(0, 0, 0, 0);
                             if (row_ok && col0 + 8 * g < N) {
-                                const uint32_t *rg = r[g >> 2] + 8 * (g & 3);
+                                const uint32_t *rg = r + 8 * g;
                                 v = dequant8<Cfg::ACC_SHIFT>(rg, sxm, sw_c + 8 * g, b_c + 8 * g);
                                 if (acc_out != nullptr) {
                                     int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N +
@@ -437,12 +439,12 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                 const int f = row;
                 const float swf = row_ok ? sw[f] : 0.0f;
                 const float bf = (row_ok && bias != nullptr) ? __half2float(bias[f]) : 0.0f;
-                const int tok_base = tn * BN + half * Cfg::EPI_COLS;
+                const int tok_base = tn * BN + cg * Cfg::EPI_COLS;
 #pragma unroll 1
                 for (int c = 0; c < NCHUNK; ++c) {
                     uint32_t r[CH];
                     __syncwarp();
-                    tmem_ld_chunk<CH>(tbase + half * Cfg::EPI_COLS + c * CH, r);
+                    tmem_ld_chunk<CH>(tbase + cg * Cfg::EPI_COLS + c * CH, r);
                     tmem_ld_wait();
                     if (c == NCHUNK - 1) {
                         tc_fence_before_sync();
@@ -458,7 +460,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                             atomicAdd(acc_buf + o, static_cast<int32_t>(r[j]));  // result unused: a reduction
                         } else {
                             const int32_t a = static_cast<int32_t>(r[j]) >> Cfg::ACC_SHIFT;
-                            Y[o] = dequant1(a, col_s[half * Cfg::EPI_COLS + c * CH + j], swf, bf);
+                            Y[o] = dequant1(a, col_s[cg * Cfg::EPI_COLS + c * CH + j], swf, bf);
                             if (acc_out != nullptr) acc_out[o] = a;
                         }
                     }
@@ -496,7 +498,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                                 const int64_t o = static_cast<int64_t>(tok) * M + f;
                                 acc_buf[o] = 0;  // zero again for the next call
                                 const int32_t a = v[j] >> Cfg::ACC_SHIFT;
-                                Y[o] = dequant1(a, col_s[half * Cfg::EPI_COLS + c * CH + j], swf, bf);
+                                Y[o] = dequant1(a, col_s[cg * Cfg::EPI_COLS + c * CH + j], swf, bf);
                                 if (acc_out != nullptr) acc_out[o] = a;
                             }
                         }
