@@ -203,6 +203,27 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// As launch_pdl, with clusters of `cluster_x` CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                               unsigned cluster_x, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int LOG2B, int BITS, bool PACKED>
 void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms, int dev,
                 uint4 *zero16, int64_t n_zero16) {
@@ -267,6 +288,7 @@ convrot_status_t rotate_quant_act_impl(const void *X, int64_t M, int64_t K, int 
 // GEMM launch plan: operand order, tile width and K split.
 struct GemmPlan {
     bool swap = false;  // feature-major (weights on the MMA's 128-row side)
+    bool pair = false;  // token-major 256 x 256 tiles on CTA pairs (cta_group::2)
     int bn = 256;       // MMA N: output features (token-major) or tokens (feature-major)
     int splits = 1;
     int64_t tiles = 0;
@@ -303,6 +325,10 @@ GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split) {
     const int64_t tiles_256 = tiles_m * ((N + 255) / 256);
     p.bn = (N >= 256 && 2 * tiles_256 > sms) ? 256 : 128;
     p.tiles = tiles_m * ((N + p.bn - 1) / p.bn);
+    // CTA pairs halve each SM's operand traffic, which pays where the main loop
+    // dominates: deep K and at least two rounds of 256 x 256 tiles
+    const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    p.pair = p.bn == 256 && K >= 1536 && pair_tiles >= sms;
     return p;
 }
 
@@ -339,10 +365,43 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, cons
     };
     const int64_t rows_a = Cfg::SWAP ? N : M, rows_b = Cfg::SWAP ? M : N;
     CR_TRY(op_map(&ta, Cfg::SWAP ? Wc : Xc, rows_a, Cfg::BM, Cfg::A4));
-    CR_TRY(op_map(&tb, Cfg::SWAP ? Xc : Wc, rows_b, Cfg::BN, Cfg::B4));
+    CR_TRY(op_map(&tb, Cfg::SWAP ? Xc : Wc, rows_b, Cfg::B_ROWS, Cfg::B4));
     if (Cfg::SWAP) ty = ta;  // stores go straight to Y
     else CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
-    const int64_t units = ((rows_a + Cfg::BM - 1) / Cfg::BM) * ((rows_b + Cfg::BN - 1) / Cfg::BN) * splits;
+    const int64_t units =
+        ((rows_a + Cfg::TILE_M - 1) / Cfg::TILE_M) * ((rows_b + Cfg::BN - 1) / Cfg::BN) * splits;
+    if (Cfg::PAIR) {
+        // persistent: one cluster of two CTAs per co-resident pair of SMs
+        static int max_clusters[kMaxDevices] = {};
+        {
+            static std::mutex mu;
+            std::lock_guard<std::mutex> lock(mu);
+            if (max_clusters[dev] == 0) {
+                cudaLaunchConfig_t occ = {};
+                occ.gridDim = dim3(2 * (info->sms / 2));
+                occ.blockDim = dim3(Cfg::NUM_THREADS);
+                occ.dynamicSmemBytes = Cfg::SMEM_BYTES;
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = 2;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                occ.attrs = attr;
+                occ.numAttrs = 1;
+                int n = 0;
+                cudaError_t e = cudaOccupancyMaxActiveClusters(&n, convrot::gemm_i8_tcgen05_kernel<Cfg>, &occ);
+                CR_REQUIRE(e == cudaSuccess && n > 0, CONVROT_ERR_CUDA, "cudaOccupancyMaxActiveClusters: %s (%d)",
+                           cudaGetErrorString(e), n);
+                max_clusters[dev] = n;
+            }
+        }
+        const int64_t clusters = units < max_clusters[dev] ? units : max_clusters[dev];
+        launch_pdl_cluster(convrot::gemm_i8_tcgen05_kernel<Cfg>, dim3(static_cast<unsigned>(2 * clusters)),
+                           dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, 2u, ta, tb, ty, static_cast<int>(rows_a),
+                           static_cast<int>(rows_b), static_cast<int>(K), sx, sw, static_cast<const __half *>(bias),
+                           static_cast<__half *>(Y), acc_out, splits, acc_buf, counters);
+        return launch_status("gemm_i8_tcgen05 (CTA pairs)");
+    }
     const int grid = static_cast<int>(units < info->sms ? units : info->sms);
     launch_pdl(convrot::gemm_i8_tcgen05_kernel<Cfg>, dim3(grid), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, ta, tb,
                ty, static_cast<int>(rows_a), static_cast<int>(rows_b), static_cast<int>(K), sx, sw,
@@ -360,9 +419,16 @@ convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const vo
     if (p.swap)
         return launch_gemm_cfg<GemmCfg<kSwapTokens, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y,
                                                                    acc_out, st, p.splits, acc_buf, counters);
-    if (p.bn == 256)
+    if (p.bn == 256) {
+        if constexpr (!X4 && !W4) {
+            if (p.pair)
+                return launch_gemm_cfg<GemmCfg<256, false, false, false, true>>(info, dev, Xc, Wc, M, N, K, sx, sw,
+                                                                                bias, Y, acc_out, st, 1, nullptr,
+                                                                                nullptr);
+        }
         return launch_gemm_cfg<GemmCfg<256, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
                                                      nullptr, nullptr);
+    }
     return launch_gemm_cfg<GemmCfg<128, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1, nullptr,
                                                  nullptr);
 }

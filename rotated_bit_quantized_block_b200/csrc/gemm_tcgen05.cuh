@@ -43,25 +43,31 @@ namespace convrot {
 // and is widened in shared memory; otherwise it is int8 loaded by TMA straight
 // into the MMA ring.  Widened bytes hold 16 * code, so the accumulator carries
 // a factor 16 per widened operand (ACC_SHIFT undoes it).
-template <int BN_, bool A4_, bool B4_, bool SWAP_ = false>
+// PAIR: a cluster of two CTAs shares each 256 x BN tile through one
+// cta_group::2 MMA (each CTA loads and keeps 128 rows of A and BN/2 rows of B).
+template <int BN_, bool A4_, bool B4_, bool SWAP_ = false, bool PAIR_ = false>
 struct GemmCfg {
-    static constexpr int BM = 128;
-    static constexpr int BN = BN_;
+    static constexpr int BM = 128;   // rows of A per CTA
+    static constexpr int BN = BN_;   // accumulator columns
     static constexpr int BK = 128;  // K elements per stage (= bytes of one int8 row segment)
     static constexpr bool A4 = A4_;
     static constexpr bool B4 = B4_;
     static constexpr bool SWAP = SWAP_;
+    static constexpr bool PAIR = PAIR_;
+    static constexpr int CTAS = PAIR ? 2 : 1;      // CTAs per tile
+    static constexpr int TILE_M = BM * CTAS;       // accumulator rows per tile
+    static constexpr int B_ROWS = BN / CTAS;       // rows of B held by one CTA
     static constexpr bool W4 = A4 || B4;          // some operand is widened by converter warps
     static constexpr bool TMA_RING = !(A4 && B4);  // some operand goes straight into the MMA ring
     static constexpr int ACC_SHIFT = (A4 ? 4 : 0) + (B4 ? 4 : 0);
     static constexpr int A_BYTES = BM * BK;
-    static constexpr int B_BYTES = BN * BK;
+    static constexpr int B_BYTES = B_ROWS * BK;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int PA_BYTES = A4 ? A_BYTES / 2 : 0;
     static constexpr int PB_BYTES = B4 ? B_BYTES / 2 : 0;
     static constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
     static constexpr int PSTAGES = !W4 ? 0 : (!SWAP && BN == 256 ? 3 : 4);
-    static constexpr int CONV_ROWS = (A4 ? BM : 0) + (B4 ? BN : 0);  // rows widened per stage
+    static constexpr int CONV_ROWS = (A4 ? BM : 0) + (B4 ? B_ROWS : 0);  // rows widened per stage
     // arrivals completing an MMA stage: the producer (TMA bytes) and/or the 128 converter threads
     static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + (W4 ? 128 : 0);
     static constexpr int TMEM_COLS = 2 * BN;
@@ -87,8 +93,9 @@ struct GemmCfg {
     static constexpr int NUM_BARRIERS = 2 * STAGES + FIXED_BARRIERS;
     static constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * STAGE_BYTES + PSTAGES * PSTAGE_BYTES +
                                       OUT_BYTES + SCALE_BYTES + NUM_BARRIERS * 8 + 16;
-    static constexpr uint32_t IDESC = idesc_i8(BM, BN);
+    static constexpr uint32_t IDESC = idesc_i8(TILE_M, BN);
     static_assert(STAGES >= 2, "pipeline depth");
+    static_assert(!PAIR || (!SWAP && !A4 && !B4 && BN == 256), "CTA pairs: token-major W8A8, 256-wide tiles");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(SWAP ? (BN == 32 || BN == 64 || BN == 128 || BN == 256) : (BN % 64 == 0 && BN >= 64 && BN <= 256),
                   "tile width");
@@ -184,9 +191,14 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     volatile int *s_last = reinterpret_cast<volatile int *>(tmem_slot + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
+    const int tiles_m = (M + Cfg::TILE_M - 1) / Cfg::TILE_M, tiles_n = (N + BN - 1) / BN;
     const int num_tiles = tiles_m * tiles_n;
     const int num_kb = K / Cfg::BK;
+    // CTA pairs: both CTAs of a cluster walk the same tiles; rank 0 issues the MMAs
+    const uint32_t rank = Cfg::PAIR ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int first_unit = Cfg::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int unit_stride = Cfg::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     // split K (feature-major only): work unit u is K slice (u % splits) of tile (u / splits)
     const int num_units = num_tiles * splits;
     auto unit_tile = [&](int u) { return u / splits; };
@@ -204,7 +216,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tmem_full[i], 1);
-            mbar_init(&tmem_empty[i], 32 * Cfg::EPI_WARPS);
+            mbar_init(&tmem_empty[i], Cfg::CTAS * 32 * Cfg::EPI_WARPS);  // every epilogue thread of the tile
         }
         mbar_init(drain, 1);
         mbar_init(scale_ready, 32 * Cfg::EPI_WARPS);
@@ -220,11 +232,17 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         if (!Cfg::SWAP) tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-        tmem_relinquish();
+        if (Cfg::PAIR) {
+            tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
+    if (Cfg::PAIR) cluster_sync();  // the peer's barriers are initialised before any remote use
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
     pdl_wait();  // the codes, scales and split-K buffers may come from the previous kernel
@@ -243,7 +261,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             for (int i = 0; i < STAGES; ++i) filled[i] = false;
             for (int i = 0; i < PSTAGES; ++i) pfilled[i] = false;
             bool ok = true;
-            for (int unit = blockIdx.x; ok && unit < num_units; unit += gridDim.x) {
+            for (int unit = first_unit; ok && unit < num_units; unit += unit_stride) {
                 const int tile = unit_tile(unit);
                 const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
                 for (int kb = unit_kb0(unit); kb < unit_kb1(unit); ++kb) {
@@ -253,9 +271,19 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                             break;
                         }
                         uint8_t *dst = ring + s * Cfg::STAGE_BYTES;
-                        mbar_arrive_expect_tx(&full[s], (Cfg::A4 ? 0 : Cfg::A_BYTES) + (Cfg::B4 ? 0 : Cfg::B_BYTES));
-                        if (!Cfg::A4) tma_load_2d(dst, &tmA, &full[s], kb * Cfg::BK, tm * BM);
-                        if (!Cfg::B4) tma_load_2d(dst + Cfg::A_BYTES, &tmB, &full[s], kb * Cfg::BK, tn * BN);
+                        if (Cfg::PAIR) {
+                            // both CTAs' bytes land on the even CTA's barrier
+                            if (leader) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+                            const uint32_t bar = cluster_addr(&full[s], 0);
+                            tma_load_2d_pair(dst, &tmA, bar, kb * Cfg::BK, tm * Cfg::TILE_M + rank * BM);
+                            tma_load_2d_pair(dst + Cfg::A_BYTES, &tmB, bar, kb * Cfg::BK,
+                                             tn * BN + rank * Cfg::B_ROWS);
+                        } else {
+                            mbar_arrive_expect_tx(&full[s],
+                                                  (Cfg::A4 ? 0 : Cfg::A_BYTES) + (Cfg::B4 ? 0 : Cfg::B_BYTES));
+                            if (!Cfg::A4) tma_load_2d(dst, &tmA, &full[s], kb * Cfg::BK, tm * BM);
+                            if (!Cfg::B4) tma_load_2d(dst + Cfg::A_BYTES, &tmB, &full[s], kb * Cfg::BK, tn * BN);
+                        }
                         filled[s] = true;
                         last_parity[s] = ph;
                         if (++s == STAGES) {
@@ -282,20 +310,28 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                 }
             }
             // no bulk copy may still be writing shared memory when the CTA exits
-            // (an MMA stage also waits for its converters when an operand is widened)
-            for (int i = 0; i < STAGES; ++i)
-                if (filled[i]) mbar_wait_drain(&full[i], last_parity[i]);
+            // (an MMA stage also waits for its converters when an operand is widened;
+            // the odd CTA of a pair sees its copies complete when the MMA frees the stage)
+            for (int i = 0; i < STAGES; ++i) {
+                if (!filled[i]) continue;
+                if (Cfg::PAIR && !leader) mbar_wait_drain(&empty[i], last_parity[i]);
+                else mbar_wait_drain(&full[i], last_parity[i]);
+            }
             for (int i = 0; i < PSTAGES; ++i)
                 if (pfilled[i]) mbar_wait_drain(&pfull[i], plast_parity[i]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (Cfg::PAIR && !leader) {
+            // the even CTA issues the pair's MMAs; wait until they have all completed
+            // (they read this CTA's shared memory)
+            if (lane == 0) mbar_wait_drain(drain, 0);
+        } else if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
             int local = 0;
-            for (int unit = blockIdx.x; ok && unit < num_units; unit += gridDim.x, ++local) {
+            for (int unit = first_unit; ok && unit < num_units; unit += unit_stride, ++local) {
                 const int acc = local & 1;
                 const uint32_t acc_ph = (local >> 1) & 1;
                 if (!mbar_wait(&tmem_empty[acc], acc_ph ^ 1, abort)) break;
@@ -312,18 +348,27 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     const uint32_t b_addr = a_addr + Cfg::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < Cfg::BK / 32; ++kk) {
-                        umma_i8(d_tmem, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
-                                Cfg::IDESC, (kb != kb0) || (kk != 0));
+                        if (Cfg::PAIR)
+                            umma_i8_pair(d_tmem, smem_desc_k_sw128(a_addr + 32 * kk),
+                                         smem_desc_k_sw128(b_addr + 32 * kk), Cfg::IDESC, (kb != kb0) || (kk != 0));
+                        else
+                            umma_i8(d_tmem, smem_desc_k_sw128(a_addr + 32 * kk), smem_desc_k_sw128(b_addr + 32 * kk),
+                                    Cfg::IDESC, (kb != kb0) || (kk != 0));
                     }
-                    umma_commit(&empty[s]);
+                    if (Cfg::PAIR) umma_commit_pair(&empty[s], 3);  // frees the stage in both CTAs
+                    else umma_commit(&empty[s]);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1;
                     }
                 }
-                if (ok) umma_commit(&tmem_full[acc]);
+                if (ok) {
+                    if (Cfg::PAIR) umma_commit_pair(&tmem_full[acc], 3);
+                    else umma_commit(&tmem_full[acc]);
+                }
             }
-            umma_commit(drain);
+            if (Cfg::PAIR) umma_commit_pair(drain, 3);
+            else umma_commit(drain);
             mbar_wait_drain(drain, 0);
         }
     } else if (warp < Cfg::FIRST_CONV_WARP) {
@@ -351,10 +396,10 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         };
         float next_w;
         __half next_b;
-        load_scales(unit_tile(blockIdx.x < num_units ? blockIdx.x : 0), next_w, next_b);
+        load_scales(unit_tile(first_unit < num_units ? first_unit : 0), next_w, next_b);
         int local = 0;
         int n_split_units = 0;  // split units handled so far (parity of the split-K barriers)
-        for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++local) {
+        for (int unit = first_unit; unit < num_units; unit += unit_stride, ++local) {
             const int tile = unit_tile(unit);
             const int acc = local & 1;
             const uint32_t acc_ph = (local >> 1) & 1;
@@ -368,9 +413,9 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             }
             mbar_arrive(scale_ready);
             if (!mbar_wait(scale_ready, local & 1, abort)) break;
-            load_scales(unit + gridDim.x < num_units ? unit_tile(unit + gridDim.x) : num_tiles, next_w, next_b);
+            load_scales(unit + unit_stride < num_units ? unit_tile(unit + unit_stride) : num_tiles, next_w, next_b);
             const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
-            const int row0 = tm * BM + q * 32;
+            const int row0 = tm * Cfg::TILE_M + static_cast<int>(rank) * BM + q * 32;
             const int row = row0 + lane;
             const bool row_ok = row < M;
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
@@ -393,7 +438,8 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     if (c == NCHUNK - 1) {
                         // every TMEM read of this unit by this thread is complete
                         tc_fence_before_sync();
-                        mbar_arrive(&tmem_empty[acc]);
+                        if (Cfg::PAIR) mbar_arrive_cluster(cluster_addr(&tmem_empty[acc], 0));
+                        else mbar_arrive(&tmem_empty[acc]);
                     }
                     const int col0 = tn * BN + col_local;
                     if (row0 >= M || col0 >= N) continue;  // whole box outside Y (warp-uniform)
@@ -514,7 +560,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         int ps = 0, us = 0;
         uint32_t pph = 0, uph = 0;
         bool ok = true;
-        for (int unit = blockIdx.x; ok && unit < num_units; unit += gridDim.x) {
+        for (int unit = first_unit; ok && unit < num_units; unit += unit_stride) {
             for (int kb = unit_kb0(unit); kb < unit_kb1(unit); ++kb) {
                 if (!mbar_wait(&pfull[ps], pph, abort) || !mbar_wait(&empty[us], uph ^ 1, abort)) {
                     ok = false;
@@ -546,9 +592,11 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     }
 
     __syncthreads();
+    if (Cfg::PAIR) cluster_sync();  // neither CTA leaves while its peer may still signal it
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+        if (Cfg::PAIR) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+        else tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
 }
 

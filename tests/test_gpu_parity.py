@@ -209,6 +209,8 @@ def run_gemm(qx, sx, qw, sw, bias, bits):
 GEMM_CASES = [
     (64, 256, 256), (1, 8, 128), (7, 24, 384), (130, 264, 640), (300, 1000, 1024),
     (256, 512, 4096), (129, 3072, 1024), (1000, 1536, 6144), (517, 4096, 256),
+    # 256-wide tiles on CTA pairs, ragged in M and N, one and several K steps
+    (1300, 2000, 384), (2600, 1032, 128),
 ]
 
 
