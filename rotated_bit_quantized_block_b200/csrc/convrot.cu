@@ -420,11 +420,10 @@ convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const vo
         return launch_gemm_cfg<GemmCfg<kSwapTokens, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y,
                                                                    acc_out, st, p.splits, acc_buf, counters);
     if (p.bn == 256) {
-        if constexpr (!X4 && !W4) {
+        if constexpr (!X4) {
             if (p.pair)
-                return launch_gemm_cfg<GemmCfg<256, false, false, false, true>>(info, dev, Xc, Wc, M, N, K, sx, sw,
-                                                                                bias, Y, acc_out, st, 1, nullptr,
-                                                                                nullptr);
+                return launch_gemm_cfg<GemmCfg<256, false, W4, false, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias,
+                                                                             Y, acc_out, st, 1, nullptr, nullptr);
         }
         return launch_gemm_cfg<GemmCfg<256, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
                                                      nullptr, nullptr);

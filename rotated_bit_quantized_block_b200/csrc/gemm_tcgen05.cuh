@@ -66,10 +66,11 @@ struct GemmCfg {
     static constexpr int PA_BYTES = A4 ? A_BYTES / 2 : 0;
     static constexpr int PB_BYTES = B4 ? B_BYTES / 2 : 0;
     static constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
-    static constexpr int PSTAGES = !W4 ? 0 : (!SWAP && BN == 256 ? 3 : 4);
+    static constexpr int PSTAGES = !W4 ? 0 : (!SWAP && BN == 256 && !PAIR ? 3 : 4);
     static constexpr int CONV_ROWS = (A4 ? BM : 0) + (B4 ? B_ROWS : 0);  // rows widened per stage
-    // arrivals completing an MMA stage: the producer (TMA bytes) and/or the 128 converter threads
-    static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + (W4 ? 128 : 0);
+    // arrivals completing an MMA stage: the producer (TMA bytes) and/or the four
+    // converter warps (of both CTAs of a pair)
+    static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + (W4 ? 4 * CTAS : 0);
     static constexpr int TMEM_COLS = 2 * BN;
     // epilogue warps: per TMEM lane quarter, EPI_WARPS / 4 warps split the columns
     // (token-major: four, so that enough warps hide the dequant's latencies)
@@ -95,12 +96,19 @@ struct GemmCfg {
                                       OUT_BYTES + SCALE_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t IDESC = idesc_i8(TILE_M, BN);
     static_assert(STAGES >= 2, "pipeline depth");
-    static_assert(!PAIR || (!SWAP && !A4 && !B4 && BN == 256), "CTA pairs: token-major W8A8, 256-wide tiles");
+    static_assert(!PAIR || (!SWAP && !A4 && BN == 256), "CTA pairs: token-major, int8 A, 256-wide tiles");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(SWAP ? (BN == 32 || BN == 64 || BN == 128 || BN == 256) : (BN % 64 == 0 && BN >= 64 && BN <= 256),
                   "tile width");
     static_assert(EPI_COLS % CHUNK == 0, "epilogue chunking");
 };
+
+// Bounded wait taken by every lane of a warp: true only if it succeeded for
+// all of them, so that a timeout leaves the warp converged (the callers then
+// use warp-collective instructions).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
 
 // Bounded wait used while draining: ignores the abort flag, still time-limited.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
@@ -273,11 +281,14 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                         uint8_t *dst = ring + s * Cfg::STAGE_BYTES;
                         if (Cfg::PAIR) {
                             // both CTAs' bytes land on the even CTA's barrier
-                            if (leader) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+                            if (leader)
+                                mbar_arrive_expect_tx(&full[s],
+                                                      2 * (Cfg::A_BYTES + (Cfg::B4 ? 0 : Cfg::B_BYTES)));
                             const uint32_t bar = cluster_addr(&full[s], 0);
                             tma_load_2d_pair(dst, &tmA, bar, kb * Cfg::BK, tm * Cfg::TILE_M + rank * BM);
-                            tma_load_2d_pair(dst + Cfg::A_BYTES, &tmB, bar, kb * Cfg::BK,
-                                             tn * BN + rank * Cfg::B_ROWS);
+                            if (!Cfg::B4)
+                                tma_load_2d_pair(dst + Cfg::A_BYTES, &tmB, bar, kb * Cfg::BK,
+                                                 tn * BN + rank * Cfg::B_ROWS);
                         } else {
                             mbar_arrive_expect_tx(&full[s],
                                                   (Cfg::A4 ? 0 : Cfg::A_BYTES) + (Cfg::B4 ? 0 : Cfg::B_BYTES));
@@ -299,7 +310,9 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                         uint8_t *dst = pring + ps * Cfg::PSTAGE_BYTES;
                         mbar_arrive_expect_tx(&pfull[ps], Cfg::PSTAGE_BYTES);
                         if (Cfg::A4) tma_load_2d(dst, &tmA, &pfull[ps], kb * (Cfg::BK / 2), tm * BM);
-                        if (Cfg::B4) tma_load_2d(dst + Cfg::PA_BYTES, &tmB, &pfull[ps], kb * (Cfg::BK / 2), tn * BN);
+                        if (Cfg::B4)
+                            tma_load_2d(dst + Cfg::PA_BYTES, &tmB, &pfull[ps], kb * (Cfg::BK / 2),
+                                        tn * BN + rank * Cfg::B_ROWS);
                         pfilled[ps] = true;
                         plast_parity[ps] = pph;
                         if (++ps == PSTAGES) {
@@ -403,16 +416,16 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             const int tile = unit_tile(unit);
             const int acc = local & 1;
             const uint32_t acc_ph = (local >> 1) & 1;
-            if (!mbar_wait(&tmem_full[acc], acc_ph, abort)) break;
+            if (!mbar_wait_warp(&tmem_full[acc], acc_ph, abort)) break;
             tc_fence_after_sync();
             // every epilogue thread is done with the previous unit's scales
-            if (local > 0 && !mbar_wait(scale_free, (local - 1) & 1, abort)) break;
+            if (local > 0 && !mbar_wait_warp(scale_free, (local - 1) & 1, abort)) break;
             if (scol < BN) {
                 col_s[scol] = next_w;
                 bias_s[scol] = next_b;
             }
             mbar_arrive(scale_ready);
-            if (!mbar_wait(scale_ready, local & 1, abort)) break;
+            if (!mbar_wait_warp(scale_ready, local & 1, abort)) break;
             load_scales(unit + unit_stride < num_units ? unit_tile(unit + unit_stride) : num_tiles, next_w, next_b);
             const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
             const int row0 = tm * Cfg::TILE_M + static_cast<int>(rank) * BM + q * 32;
@@ -526,7 +539,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                         *s_last = last;
                         mbar_arrive(decided);
                     }
-                    if (!mbar_wait(decided, n_split_units & 1, abort)) break;
+                    if (!mbar_wait_warp(decided, n_split_units & 1, abort)) break;
                     ++n_split_units;
                     if (*s_last != 0 && row_ok) {
 #pragma unroll 1
@@ -562,7 +575,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         bool ok = true;
         for (int unit = first_unit; ok && unit < num_units; unit += unit_stride) {
             for (int kb = unit_kb0(unit); kb < unit_kb1(unit); ++kb) {
-                if (!mbar_wait(&pfull[ps], pph, abort) || !mbar_wait(&empty[us], uph ^ 1, abort)) {
+                if (!mbar_wait_warp(&pfull[ps], pph, abort) || !mbar_wait_warp(&empty[us], uph ^ 1, abort)) {
                     ok = false;
                     break;
                 }
@@ -576,8 +589,13 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     const uint2 p = *reinterpret_cast<const uint2 *>(src + rr * 64 + piece * 8);
                     *reinterpret_cast<uint4 *>(dst + rr * 128 + ((piece ^ (rr & 7)) << 4)) = widen_int4x16(p);
                 }
+                // the widened bytes are visible to the tensor core before the stage is signalled
                 fence_proxy_async_smem();
-                mbar_arrive(&full[us]);
+                __syncwarp();
+                if (lane == 0) {
+                    if (Cfg::PAIR) mbar_arrive_cluster(cluster_addr(&full[us], 0));
+                    else mbar_arrive(&full[us]);
+                }
                 mbar_arrive(&pempty[ps]);
                 if (++ps == PSTAGES) {
                     ps = 0;

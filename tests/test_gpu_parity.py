@@ -209,7 +209,7 @@ def run_gemm(qx, sx, qw, sw, bias, bits):
 GEMM_CASES = [
     (64, 256, 256), (1, 8, 128), (7, 24, 384), (130, 264, 640), (300, 1000, 1024),
     (256, 512, 4096), (129, 3072, 1024), (1000, 1536, 6144), (517, 4096, 256),
-    # 256-wide tiles on CTA pairs, ragged in M and N, one and several K steps
+    # 256-wide tiles, ragged in M and N, one and several K steps
     (1300, 2000, 384), (2600, 1032, 128),
 ]
 
@@ -345,3 +345,45 @@ def test_linear_split_k_bit_exact(M, N, K, bits):
     qw = unpack(host(Wq), bits)
     yr = oracle.gemm_dequant(qx, sx, qw, host(sw), bias)
     assert np.array_equal(outs[0].view(np.uint16), yr.view(np.uint16))
+
+
+def pair_rows(M):
+    """Rows to check on a 256-row-tile GEMM: both 128-row halves of the first
+    and last tiles, every tile's first row, and the ragged tail."""
+    rows = {0, 127, 128, 255, M - 1, M - 2}
+    rows |= set(range(0, M, 256)) | set(range(128, M, 256))
+    rows |= set(range(max(0, M - 140), M, 7))
+    return np.array(sorted(r for r in rows if 0 <= r < M))
+
+
+@pytest.mark.parametrize("M,N,K", [(2700, 4000, 1536), (4100, 2056, 2048)])
+def test_gemm_pair_tiles_bit_exact_sampled(M, N, K):
+    """Shapes the plan runs on CTA pairs (deep K, many 256 x 256 tiles), ragged in M and N."""
+    qx, sx, qw, sw = oracle_codes(M, N, K, 128, 8, seed=M + K)
+    bias = wl.bias(N, seed=5)
+    y, acc = run_gemm(qx, sx, qw, sw, bias, 8)
+    rows = pair_rows(M)
+    yr, accr = oracle.gemm_dequant(qx[rows], sx[rows], qw, sw, bias, want_acc=True)
+    assert np.array_equal(acc[rows], accr)
+    assert np.array_equal(y[rows].view(np.uint16), yr.view(np.uint16))
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_linear_pair_tiles_bit_exact_sampled(bits):
+    """The linear on CTA pairs (int8 activations, int8 or widened int4 weights):
+    the output equals the oracle's GEMM of the workspace's codes on sampled rows."""
+    M, N, K = 2700, 4000, 1536
+    X = wl.activations(M, K, 0.01, 30.0, seed=17)
+    W = wl.weight(N, K, 0.02, seed=18)
+    bias = wl.bias(N, seed=19)
+    Wq, sw = cr.convrot_quantize_weight(dev(W), 128, bits, cr.CLIP_ABSMAX)
+    fn = cr.convrot_linear_w8a8 if bits == 8 else cr.convrot_linear_w4a4
+    ws = torch.empty(cr.convrot_linear_workspace_bytes(M, K, N, bits), dtype=torch.uint8, device="cuda")
+    y = host(fn(dev(X), Wq, sw, 128, bias=dev(bias), workspace=ws))
+    raw = host(ws)
+    qx = raw[: M * K].view(np.int8).reshape(M, K)
+    off = (M * K + 255) // 256 * 256
+    sx = raw[off: off + 4 * M].view(np.float32)
+    rows = pair_rows(M)
+    yr = oracle.gemm_dequant(qx[rows], sx[rows], unpack(host(Wq), bits), host(sw), bias)
+    assert np.array_equal(y[rows].view(np.uint16), yr.view(np.uint16))
