@@ -81,6 +81,7 @@ def _load():
         "oracle_quant_error": (f64, [P, i64, f32, i32]),
         "oracle_alpha": (f32, [i32]),
         "oracle_quantize_weight": (i32, [P, i32, i64, i64, i32, i32, i32, P, P, P, P]),
+        "oracle_quantize_weight_tensorwise": (i32, [P, i32, i64, i64, i32, i32, i32, P, P, P, P]),
         "oracle_rotate_quant_act": (i32, [P, i64, i64, i32, i32, P, P]),
         "oracle_pack_int4": (i32, [P, i64, P]),
         "oracle_unpack_int4": (i32, [P, i64, P]),
@@ -205,6 +206,28 @@ def quantize_weight(W, b: int, bits: int, clip_mode: int = CLIP_MSE, dtype: int 
                                         _ptr(codes), _ptr(scales), _ptr(aidx), _ptr(errs))
     _check(rc, "quantize_weight")
     return (codes, scales, aidx, errs) if want_errs else (codes, scales, aidx)
+
+
+def quantize_weight_tensorwise(W, b: int, bits: int, clip_mode: int = CLIP_MSE, dtype: int = DTYPE_F16,
+                               want_errs: bool = False):
+    """Tensor-wise variant of the converter: one scale for the whole weight
+    tensor (salahadawi.com "Explanation of INT8 ConvRot", "8-bit INT type
+    models" table, Tensor-wise scaling; civarchive.com release, downloads
+    table, int8_tensorwise).  Returns ``(codes int8 N x K, scales fp32 N (all
+    equal), alpha_idx int[, errs 51])``.
+    """
+    if isinstance(W, np.ndarray) and W.dtype == np.float16:
+        W = W.view(np.uint16)
+    W = np.ascontiguousarray(W)
+    N, K = W.shape
+    codes = np.empty((N, K), dtype=np.int8)
+    scales = np.empty(N, dtype=np.float32)
+    aidx = np.zeros(1, dtype=np.int32)
+    errs = np.empty(MSE_GRID, dtype=np.float64) if want_errs else None
+    rc = _load().oracle_quantize_weight_tensorwise(_ptr(W), dtype, N, K, int(b), bits, clip_mode,
+                                                   _ptr(codes), _ptr(scales), _ptr(aidx), _ptr(errs))
+    _check(rc, "quantize_weight_tensorwise")
+    return (codes, scales, int(aidx[0]), errs) if want_errs else (codes, scales, int(aidx[0]))
 
 
 def rotate_quant_act(X_f16, b: int, bits: int):

@@ -314,6 +314,80 @@ int oracle_quantize_weight(const void *W, int dtype, int64_t N, int64_t K, int b
     return bad ? ORACLE_ERR_ARG : ORACLE_OK;
 }
 
+/* Tensor-wise variant of the converter (salahadawi.com "Explanation of INT8
+ * ConvRot", "8-bit INT type models" table: Tensor-wise scaling, one scale per
+ * weight tensor; civarchive.com release, downloads table: an int8_tensorwise
+ * ConvRot file).  Same rotation and code rule as oracle_quantize_weight, but
+ * one scale for all rows: s = fp32(fp32(alpha * max over the tensor of |W~|) /
+ * qmax), with alpha from the same grid.  In MSE mode alpha minimises the
+ * total squared error of the tensor, the rows' float64 errors summed in row
+ * order (first strict minimum from alpha = 1).  `scales` receives s for every
+ * row, `errs` (if given) the tensor's error for each grid point. */
+int oracle_quantize_weight_tensorwise(const void *W, int dtype, int64_t N, int64_t K, int b, int bits,
+                                      int clip_mode, int8_t *codes, float *scales, int32_t *alpha_idx,
+                                      double *errs)
+{
+    if (!W || !codes || !scales || N < 0 || K <= 0 || !is_pow2(b) || K % b) return ORACLE_ERR_ARG;
+    if (bits != 8 && bits != 4) return ORACLE_ERR_ARG;
+    if (clip_mode != ORACLE_CLIP_ABSMAX && clip_mode != ORACLE_CLIP_MSE) return ORACLE_ERR_ARG;
+    double *Rb = (double *)malloc(sizeof(double) * (size_t)b * b);
+    float *w = (float *)malloc(sizeof(float) * (size_t)(N > 0 ? N : 1) * (size_t)K);
+    float *row_max = (float *)malloc(sizeof(float) * (size_t)(N > 0 ? N : 1));
+    oracle_hadamard(b, Rb);
+    int64_t n;
+    int bad = 0;
+    /* step 1: every row rotated and rounded to fp32, and its absmax */
+#pragma omp parallel for schedule(dynamic, 4) reduction(| : bad)
+    for (n = 0; n < N; ++n) {
+        double *src = (double *)malloc(sizeof(double) * (size_t)K);
+        double *rot = (double *)malloc(sizeof(double) * (size_t)K);
+        if (dtype == ORACLE_DTYPE_F32)
+            bad |= oracle_decode((const float *)W + n * K, dtype, K, src);
+        else
+            bad |= oracle_decode((const uint16_t *)W + n * K, dtype, K, src);
+        rotate_row(src, K, b, Rb, rot);
+        for (int64_t k = 0; k < K; ++k) w[n * K + k] = (float)rot[k];
+        row_max[n] = row_absmax(w + n * K, K);
+        free(src);
+        free(rot);
+    }
+    /* step 2: the tensor's absmax */
+    float a = 0.0f;
+    for (n = 0; n < N; ++n) a = row_max[n] > a ? row_max[n] : a;
+    /* step 3: the clip choice */
+    int n_alpha = clip_mode == ORACLE_CLIP_MSE ? ORACLE_MSE_GRID : 1;
+    double *row_err = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1) * ORACLE_MSE_GRID);
+#pragma omp parallel for schedule(dynamic, 4)
+    for (n = 0; n < N; ++n)
+        for (int i = 0; i < n_alpha; ++i)
+            row_err[n * ORACLE_MSE_GRID + i] = oracle_quant_error(w + n * K, K, oracle_scale(a, oracle_alpha(i), bits), bits);
+    int best = 0;
+    double best_err = INFINITY;
+    for (int i = 0; i < n_alpha; ++i) {
+        double e = 0.0;
+        for (n = 0; n < N; ++n) e += row_err[n * ORACLE_MSE_GRID + i];
+        if (errs) errs[i] = e;
+        if (e < best_err) {
+            best_err = e;
+            best = i;
+        }
+    }
+    /* step 4: every row quantized with the one scale */
+    float s = oracle_scale(a, oracle_alpha(best), bits);
+    float inv = oracle_inv_scale(s);
+#pragma omp parallel for schedule(static)
+    for (n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) codes[n * K + k] = (int8_t)oracle_quantize_value(w[n * K + k], inv, bits);
+        scales[n] = s;
+    }
+    if (alpha_idx) *alpha_idx = best;
+    free(row_err);
+    free(row_max);
+    free(w);
+    free(Rb);
+    return bad ? ORACLE_ERR_ARG : ORACLE_OK;
+}
+
 /* Online activation path: X (M x K fp16) -> X.R rounded to fp32 -> per-token
  * absmax scale s_x[m] = fp32(amax / qmax) -> codes (unpacked int8). */
 int oracle_rotate_quant_act(const uint16_t *X, int64_t M, int64_t K, int b, int bits, int8_t *codes,

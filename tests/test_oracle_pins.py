@@ -439,3 +439,69 @@ def test_epilogue_multiply_add_rounds_once():
         t = np.float32(np.float32(acc) * sx)  # IEEE fp32 product
         exact = Fraction(float(t)) * Fraction(float(sw)) + Fraction(float(bias))
         assert _is_nearest_f32(exact, got), (acc, sx, sw, bias)
+
+
+# ----------------------------------------------------------------------------- tensor-wise variant
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_tensorwise_mse_matches_bruteforce_with_library_quantizer(bits):
+    """One scale for the tensor: brute force over the grid with torch's
+    fake-quant routine on the whole (unrotated, b = 1) tensor; the oracle's
+    pick is the first strict minimiser and its per-alpha errors agree."""
+    rng = np.random.default_rng(10 + bits)
+    W = rng.standard_t(2, size=(5, 64)).astype(np.float16)
+    codes, scales, aidx, errs = oracle.quantize_weight_tensorwise(W, 1, bits, oracle.CLIP_MSE, want_errs=True)
+    qmax, qmin = oracle.qmax(bits), oracle.qmin(bits)
+    w32 = W.astype(np.float32)
+    amax = np.float32(np.max(np.abs(w32)))
+    brute = []
+    for i in range(oracle.MSE_GRID):
+        a = np.float32(np.float32(100 - i) / np.float32(100))
+        s = np.float32(np.float32(a * amax) / np.float32(qmax))
+        deq = torch.fake_quantize_per_tensor_affine(torch.from_numpy(w32), float(s), 0, qmin, qmax)
+        brute.append(float(np.sum((w32.astype(np.float64) - deq.numpy().astype(np.float64)) ** 2)))
+    brute = np.array(brute)
+    assert np.allclose(errs, brute, rtol=1e-5, atol=1e-12)
+    assert errs[aidx] <= brute.min() * (1 + 1e-5) + 1e-12
+    assert np.all(errs[:aidx] > errs[aidx])
+    s = scales[0].astype(np.float64)
+    assert np.all(scales == scales[0])
+    clipped = np.abs(w32) > s * qmax
+    assert np.all(np.isin(codes[clipped], [qmin, qmax, -qmax]))
+    assert np.all(np.abs(w32[~clipped] - s * codes[~clipped]) <= s * 0.5 * (1 + 1e-5))
+
+
+def test_tensorwise_absmax_scale_and_codes_from_a_dense_rotation():
+    """Absmax mode against a dense float64 rotation (scipy's Hadamard): the
+    scale is the tensor's max |W R| / qmax and the codes are rne(x * (1/s))."""
+    b, K = 64, 256
+    W = workloads.weight(8, K, 0.02, 21)
+    R = scipy.linalg.block_diag(*([scipy.linalg.hadamard(b) / math.sqrt(b)] * (K // b)))
+    WR = (W.astype(np.float64) @ R).astype(np.float32)
+    s_ref = np.float32(np.float32(1.0 * np.max(np.abs(WR))) / np.float32(127))
+    codes, scales, aidx = oracle.quantize_weight_tensorwise(W, b, 8, oracle.CLIP_ABSMAX)
+    assert aidx == 0
+    assert np.all(scales == scales[0])
+    assert abs(float(scales[0]) - float(s_ref)) <= 1e-6 * float(s_ref)
+    inv = np.float64(np.float32(1.0) / scales[0])
+    ref = np.clip(np.rint(WR.astype(np.float64) * inv), -127, 127)
+    d = np.abs(codes.astype(np.int32) - ref.astype(np.int32))
+    assert d.max() <= 1 and np.count_nonzero(d) <= 1e-3 * d.size
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("clip", [0, 1])
+def test_tensorwise_single_row_is_rowwise(bits, clip):
+    """With one row the tensor is the row: both converters agree exactly."""
+    W = workloads.weight(1, 512, 0.02, 5)
+    c1, s1, a1 = oracle.quantize_weight(W, 128, bits, clip)
+    c2, s2, a2 = oracle.quantize_weight_tensorwise(W, 128, bits, clip)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2) and int(a1[0]) == a2
+
+
+def test_tensorwise_absmax_scale_is_the_largest_row_scale():
+    """Rounding is monotone, so max_n fp32(amax_n / qmax) = fp32(max_n amax_n / qmax)."""
+    W = workloads.weight(16, 256, 0.02, 23)
+    _, s_rows, _ = oracle.quantize_weight(W, 64, 4, oracle.CLIP_ABSMAX)
+    _, s_t, _ = oracle.quantize_weight_tensorwise(W, 64, 4, oracle.CLIP_ABSMAX)
+    assert np.all(s_t == s_rows.max())
