@@ -174,8 +174,8 @@ class Replica:
             X, W, _ = wl.linear_inputs(w, i, replica=replica)
             Xd = torch.from_numpy(X).to(device)
             Wd = torch.from_numpy(W).to(device)
-            Wq, sw = cr.convrot_quantize_weight(Wd, w.block, w.bits, cr.CLIP_MSE)
-            need = cr.convrot_linear_workspace_bytes(w.M, lin.K, lin.N, w.bits)
+            Wq, sw = cr.convrot_quantize_weight(Wd, w.block, w.bits_of(lin), cr.CLIP_MSE)
+            need = cr.convrot_linear_workspace_bytes(w.M, lin.K, lin.N, w.bits_of(lin))
             self.items.append({
                 "lin": lin, "X": Xd, "Xhost": torch.from_numpy(X).pin_memory(), "Wq": Wq, "sw": sw,
                 "Y": torch.empty((w.M, lin.N), dtype=torch.float16, device=device),
@@ -202,10 +202,10 @@ def run_step(w, rep, stream, events=None):
         ws = it["ws"]
         if events is not None:
             events[i][0].record(stream)
-        cr.convrot_linear_quant_act(it["X"], w.block, w.bits, ws, stream=stream)
+        cr.convrot_linear_quant_act(it["X"], w.block, w.bits_of(lin), ws, stream=stream)
         if events is not None:
             events[i][1].record(stream)
-        cr.convrot_linear_gemm(ws, w.M, lin.K, w.bits, it["Wq"], it["sw"], None, it["Y"], stream=stream)
+        cr.convrot_linear_gemm(ws, w.M, lin.K, w.bits_of(lin), it["Wq"], it["sw"], None, it["Y"], stream=stream)
         if events is not None:
             events[i][2].record(stream)
 
@@ -213,7 +213,7 @@ def run_step(w, rep, stream, events=None):
 def run_step_linear(w, rep, stream):
     """One pass through the public linear entry point (what a user calls)."""
     for it in rep.items:
-        fn = cr.convrot_linear_w8a8 if w.bits == 8 else cr.convrot_linear_w4a4
+        fn = cr.convrot_linear_w8a8 if w.bits_of(it["lin"]) == 8 else cr.convrot_linear_w4a4
         fn(it["X"], it["Wq"], it["sw"], w.block, None, it["Y"], it["ws"], stream)
 
 
@@ -231,7 +231,7 @@ def oracle_weights(w: wl.Workload):
         weights = []
         for i in range(len(w.linears)):
             X, W, _ = wl.linear_inputs(w, i)
-            qw, sw, _ = oracle.quantize_weight(W, w.block, w.bits, oracle.CLIP_MSE)
+            qw, sw, _ = oracle.quantize_weight(W, w.block, w.bits_of(w.linears[i]), oracle.CLIP_MSE)
             weights.append((X, qw, sw))
         _ORACLE_WEIGHTS[w.name] = weights
     return _ORACLE_WEIGHTS[w.name]
@@ -247,8 +247,8 @@ def time_oracle(w: wl.Workload, budget_s: float, max_rows: int | None = None):
 
     def run(rows):
         t0 = time.perf_counter()
-        for X, qw, sw in weights:
-            oracle.linear(X[:rows], qw, sw, w.block, w.bits)
+        for lin, (X, qw, sw) in zip(w.linears, weights):
+            oracle.linear(X[:rows], qw, sw, w.block, w.bits_of(lin))
         return time.perf_counter() - t0
 
     rows = max(1, min(w.M, 2 * threads))
@@ -287,7 +287,7 @@ def reference_arm(args, w, rank, world):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * w.M / value,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8" if w.bits == 8 else "int4",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype_of(w, mma=False),
         "data": "synthetic", "config": config_of(w),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": runs[0]["threads"], "kind": "oracle",
                          "sample": f"{rows} of {w.M} tokens through every linear per step "
@@ -299,13 +299,27 @@ def reference_arm(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def widths(w: wl.Workload):
+    return sorted({w.bits_of(l) for l in w.linears}, reverse=True)
+
+
+def dtype_of(w: wl.Workload, mma: bool = True) -> str:
+    names = {8: "int8", 4: "int4 (int8 MMA)" if mma else "int4"}
+    return " / ".join(names[b] for b in widths(w))
+
+
 def config_of(w: wl.Workload):
+    if len(widths(w)) == 1:
+        width = f"W{w.bits}A{w.bits}"
+    else:
+        width = "per-layer " + ", ".join(f"{l.name} W{w.bits_of(l)}A{w.bits_of(l)}" for l in w.linears)
     return {
         "workload": f"{w.name}: " + ", ".join(f"{l.name} {l.K}->{l.N}" for l in w.linears)
-                    + f"; M={w.M} tokens; Hadamard block {w.block}; W{w.bits}A{w.bits}; "
+                    + f"; M={w.M} tokens; Hadamard block {w.block}; {width}; "
                       f"acts N(0,1) with {w.outlier_frac:.1%} outlier channels x{w.outlier_factor:g}; "
                       f"W N(0,{w.w_sigma})",
-        "M": w.M, "block": w.block, "bits": w.bits, "linears": [[l.name, l.K, l.N] for l in w.linears],
+        "M": w.M, "block": w.block, "bits": w.bits if len(widths(w)) == 1 else [w.bits_of(l) for l in w.linears],
+        "linears": [[l.name, l.K, l.N] for l in w.linears],
         "parallelism": "replicas (M-split, no collective)",
     }
 
@@ -329,7 +343,7 @@ def ours_arm(args, w, rank, world, local_rank):
     with torch.cuda.stream(stream):
         wq_ev[0].record(stream)
         for it in reps[0].items:
-            cr.convrot_quantize_weight(it["W"], w.block, w.bits, cr.CLIP_MSE, stream=stream)
+            cr.convrot_quantize_weight(it["W"], w.block, w.bits_of(it["lin"]), cr.CLIP_MSE, stream=stream)
         wq_ev[1].record(stream)
     torch.cuda.synchronize()
     weight_quant_ms = wq_ev[0].elapsed_time(wq_ev[1])
@@ -428,7 +442,7 @@ def ours_arm(args, w, rank, world, local_rank):
         # mean DRAM bytes per GEMM launch of one step, from the committed ncu capture
         "traffic": (statistics.mean(gemm_traffic.values()) if gemm_traffic else None),
         "traffic_per_linear": gemm_traffic,
-        "algorithmic_bytes_per_linear": {l.name: w.M * l.K + l.N * l.K * w.bits // 8 + 2 * w.M * l.N + 4 * w.M + 4 * l.N
+        "algorithmic_bytes_per_linear": {l.name: w.M * l.K + l.N * l.K * w.bits_of(l) // 8 + 2 * w.M * l.N + 4 * w.M + 4 * l.N
                                          for l in w.linears},
         "kernel": "gemm_i8_tcgen05 (int8 x int8 -> int32, fused dequant epilogue)",
         "peak_note": f"dense int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s",
@@ -437,7 +451,7 @@ def ours_arm(args, w, rank, world, local_rank):
         "per_linear_tops": {l.name: round(2 * w.M * l.K * l.N / (t / 1000) / 1e12, 1)
                             for l, t in zip(w.linears, per_linear_ms)},
     }
-    act_bytes = [w.M * l.K * 2 + w.M * l.K * w.bits // 8 + 4 * w.M for l in w.linears]
+    act_bytes = [w.M * l.K * 2 + w.M * l.K + 4 * w.M for l in w.linears]  # codes one byte each in the linear
     act_total_ms = sum(per_linear_act_ms)
     act_gbs = sum(act_bytes) / (act_total_ms / 1000.0) / 1e9
     act_traffic = traffic["act"]
@@ -454,7 +468,7 @@ def ours_arm(args, w, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8" if w.bits == 8 else "int4 (int8 MMA)", "data": "synthetic",
+        "vs_baseline": None, "dtype": dtype_of(w), "data": "synthetic",
         "config": dict(config_of(w), l2=f"inputs larger than L2: 2 rotating buffer sets of "
                                         f"{per_set / 2**20:.0f} MiB each (L2 {L2_BYTES >> 20} MiB)"),
         "tops": ops_step * world * args.steps / (elapsed_ms / 1000.0) / 1e12,

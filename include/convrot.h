@@ -89,6 +89,28 @@ convrot_status_t convrot_quantize_weight(const void *W, int w_dtype, int64_t N, 
                                          void *stream);
 
 /*
+ * Tensor-wise variant of the offline converter (salahadawi.com "Explanation
+ * of INT8 ConvRot", "8-bit INT type models" table: Tensor-wise scaling, one
+ * scale per weight tensor; civarchive.com release, downloads table: an
+ * int8_tensorwise ConvRot file).  Same rotation and code rule as
+ * convrot_quantize_weight; the scale is shared by all rows:
+ * s = fp32(fp32(alpha * max over the tensor of |W~|) / qmax), alpha = 1 in
+ * CONVROT_CLIP_ABSMAX mode or, in CONVROT_CLIP_MSE mode, the grid point with
+ * the smallest total squared error of the tensor (the rows' float64 errors
+ * summed in row order; first strict minimum from alpha = 1).  w_scale[N]
+ * receives s for every row, so the linears and GEMMs take the result as is.
+ *   workspace  at least convrot_tensorwise_workspace_bytes(N, clip_mode) bytes
+ *              of device memory, 16-byte aligned; its contents on return are
+ *              unspecified.
+ * Four launches on `stream` (row absmax, tensor absmax, [row errors, clip
+ * choice,] quantization); other arguments and errors as convrot_quantize_weight.
+ */
+size_t convrot_tensorwise_workspace_bytes(int64_t N, int clip_mode);
+convrot_status_t convrot_quantize_weight_tensorwise(const void *W, int w_dtype, int64_t N, int64_t K, int block,
+                                                    int bits, int clip_mode, void *Wq, float *w_scale,
+                                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Online activation quantization -- "online 8-bit activation quantization",
  * "dynamic per-operation" (civarchive ConvRot release, "Quantization recipe"),
  * with the matching rotation of "What ConvRot changes" (trellis3d.app):

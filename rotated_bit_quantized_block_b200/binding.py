@@ -24,7 +24,7 @@ EXPORTED = (
     "convrot_linear_w8a8", "convrot_linear_w4a4", "convrot_gemm_w8a8", "convrot_gemm_w4a4",
     "convrot_device_status", "convrot_status_string", "convrot_last_error", "convrot_version",
     "convrot_linear_w8a8_noalloc", "convrot_linear_quant_act", "convrot_linear_gemm",
-    "convrot_linear_workspace_bytes",
+    "convrot_linear_workspace_bytes", "convrot_tensorwise_workspace_bytes", "convrot_quantize_weight_tensorwise",
 )
 
 
@@ -53,6 +53,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
             "convrot_rotate_quant_act": (i32, [P, i64, i64, i32, i32, P, P, P]),
             "convrot_workspace_bytes": (sz, [i64, i64, i32]),
             "convrot_linear_workspace_bytes": (sz, [i64, i64, i64, i32]),
+            "convrot_tensorwise_workspace_bytes": (sz, [i64, i32]),
+            "convrot_quantize_weight_tensorwise": (i32, [P, i32, i64, i64, i32, i32, i32, P, P, P, sz, P]),
             "convrot_linear_w8a8": (i32, [P, i64, i64, P, P, i64, P, i32, P, P, sz, P]),
             "convrot_linear_w4a4": (i32, [P, i64, i64, P, P, i64, P, i32, P, P, sz, P]),
             "convrot_gemm_w8a8": (i32, [P, P, i64, P, P, i64, i64, P, P, P, P]),
@@ -121,6 +123,30 @@ def convrot_quantize_weight(W: torch.Tensor, block: int, bits: int, clip_mode: i
         w_scale = torch.empty(N, dtype=torch.float32, device=W.device)
     st = load_library().convrot_quantize_weight(_ptr(W), _TORCH_DTYPE[W.dtype], N, K, block, bits, clip_mode,
                                                 _ptr(Wq), _ptr(w_scale), _stream(stream))
+    _check(st)
+    return Wq, w_scale
+
+
+def convrot_tensorwise_workspace_bytes(N: int, clip_mode: int) -> int:
+    return int(load_library().convrot_tensorwise_workspace_bytes(N, clip_mode))
+
+
+def convrot_quantize_weight_tensorwise(W: torch.Tensor, block: int, bits: int, clip_mode: int = CLIP_MSE, Wq=None,
+                                       w_scale=None, workspace=None, stream=None):
+    """Offline rotate + clip search + quantization of W with one scale for the
+    whole tensor (w_scale holds it for every row)."""
+    _dev(W, "W")
+    N, K = W.shape
+    if Wq is None:
+        Wq = torch.empty(code_shape(N, K, bits), dtype=code_dtype(bits), device=W.device)
+    if w_scale is None:
+        w_scale = torch.empty(N, dtype=torch.float32, device=W.device)
+    if workspace is None:
+        workspace = torch.empty(max(1, convrot_tensorwise_workspace_bytes(N, clip_mode)), dtype=torch.uint8,
+                                device=W.device)
+    st = load_library().convrot_quantize_weight_tensorwise(
+        _ptr(W), _TORCH_DTYPE[W.dtype], N, K, block, bits, clip_mode, _ptr(Wq), _ptr(w_scale), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st)
     return Wq, w_scale
 

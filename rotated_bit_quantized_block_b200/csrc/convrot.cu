@@ -262,14 +262,38 @@ void dispatch_act(int log2b, const void *X, int64_t M, int64_t K, void *Xq, floa
     }
 }
 
+// Tensor-wise passes: see weight_rotate_quant_kernel (all null = row-wise).
+struct WeightPass {
+    const float *given_amax = nullptr;
+    const int *given_alpha = nullptr;
+    float *row_amax_out = nullptr;
+    double *row_err_out = nullptr;
+};
+
 template <int LOG2B>
 void launch_weight(const void *W, int dtype, int64_t N, int64_t K, int bits, int clip, void *Wq, float *ws,
-                   cudaStream_t st) {
+                   cudaStream_t st, const WeightPass &ps) {
     int R, T;
     rotate_geometry(K, &R, &T);
     const int64_t grid = (N + R - 1) / R;
     convrot::weight_rotate_quant_kernel<LOG2B><<<static_cast<unsigned>(grid), T, 0, st>>>(
-        W, dtype, N, static_cast<int>(K), R, bits, clip, Wq, ws);
+        W, dtype, N, static_cast<int>(K), R, bits, clip, Wq, ws, ps.given_amax, ps.given_alpha, ps.row_amax_out,
+        ps.row_err_out);
+}
+
+void dispatch_weight(int log2b, const void *W, int dtype, int64_t N, int64_t K, int bits, int clip, void *Wq,
+                     float *ws, cudaStream_t st, const WeightPass &ps = WeightPass()) {
+    switch (log2b) {
+        case 0: launch_weight<0>(W, dtype, N, K, bits, clip, Wq, ws, st, ps); break;
+        case 1: launch_weight<1>(W, dtype, N, K, bits, clip, Wq, ws, st, ps); break;
+        case 2: launch_weight<2>(W, dtype, N, K, bits, clip, Wq, ws, st, ps); break;
+        case 3: launch_weight<3>(W, dtype, N, K, bits, clip, Wq, ws, st, ps); break;
+        case 4: launch_weight<4>(W, dtype, N, K, bits, clip, Wq, ws, st, ps); break;
+        case 5: launch_weight<5>(W, dtype, N, K, bits, clip, Wq, ws, st, ps); break;
+        case 6: launch_weight<6>(W, dtype, N, K, bits, clip, Wq, ws, st, ps); break;
+        case 7: launch_weight<7>(W, dtype, N, K, bits, clip, Wq, ws, st, ps); break;
+        default: launch_weight<8>(W, dtype, N, K, bits, clip, Wq, ws, st, ps); break;
+    }
 }
 
 // packed: int4 codes two per byte (bits = 4 only); otherwise one byte per code.
@@ -512,18 +536,61 @@ convrot_status_t convrot_quantize_weight(const void *W, int w_dtype, int64_t N, 
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (ilog2(block)) {
-        case 0: launch_weight<0>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
-        case 1: launch_weight<1>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
-        case 2: launch_weight<2>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
-        case 3: launch_weight<3>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
-        case 4: launch_weight<4>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
-        case 5: launch_weight<5>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
-        case 6: launch_weight<6>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
-        case 7: launch_weight<7>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
-        default: launch_weight<8>(W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st); break;
-    }
+    dispatch_weight(ilog2(block), W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st);
     return launch_status("weight_rotate_quant");
+}
+
+size_t convrot_tensorwise_workspace_bytes(int64_t N, int clip_mode) {
+    if (N < 0 || (clip_mode != CONVROT_CLIP_ABSMAX && clip_mode != CONVROT_CLIP_MSE)) return 0;
+    size_t b = round256(static_cast<size_t>(N) * 4) + 256;  // row absmax, then the tensor's absmax and clip index
+    if (clip_mode == CONVROT_CLIP_MSE) b += round256(static_cast<size_t>(N) * convrot::kMseGrid * 8);
+    return b;
+}
+
+convrot_status_t convrot_quantize_weight_tensorwise(const void *W, int w_dtype, int64_t N, int64_t K, int block,
+                                                    int bits, int clip_mode, void *Wq, float *w_scale,
+                                                    void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    CR_TRY(check_shape(N, K, block, "N"));
+    CR_TRY(check_bits(bits));
+    CR_REQUIRE(w_dtype >= CONVROT_DTYPE_F16 && w_dtype <= CONVROT_DTYPE_F32, CONVROT_ERR_INVALID_ARG,
+               "w_dtype = %d is not one of fp16 / bf16 / fp32", w_dtype);
+    CR_REQUIRE(clip_mode == CONVROT_CLIP_ABSMAX || clip_mode == CONVROT_CLIP_MSE, CONVROT_ERR_INVALID_ARG,
+               "clip_mode = %d", clip_mode);
+    if (N == 0) return ok();
+    CR_REQUIRE(W && Wq && w_scale, CONVROT_ERR_INVALID_ARG, "null pointer argument");
+    CR_REQUIRE(aligned(W, 16) && aligned(Wq, 16), CONVROT_ERR_ALIGNMENT, "W and Wq must be 16-byte aligned");
+    CR_REQUIRE(aligned(w_scale, 4), CONVROT_ERR_ALIGNMENT, "w_scale must be 4-byte aligned");
+    const size_t need = convrot_tensorwise_workspace_bytes(N, clip_mode);
+    CR_REQUIRE(workspace != nullptr && workspace_bytes >= need, CONVROT_ERR_WORKSPACE,
+               "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+    CR_REQUIRE(aligned(workspace, 16), CONVROT_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *wsp = static_cast<uint8_t *>(workspace);
+    float *row_amax = reinterpret_cast<float *>(wsp);
+    float *g_amax = reinterpret_cast<float *>(wsp + round256(static_cast<size_t>(N) * 4));
+    int *g_alpha = reinterpret_cast<int *>(g_amax + 4);
+    double *row_err = reinterpret_cast<double *>(wsp + round256(static_cast<size_t>(N) * 4) + 256);
+    const int log2b = ilog2(block);
+    WeightPass stats;
+    stats.row_amax_out = row_amax;
+    dispatch_weight(log2b, W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st, stats);
+    convrot::amax_reduce_kernel<<<1, 1024, 0, st>>>(row_amax, N, g_amax);
+    WeightPass quant;
+    quant.given_amax = g_amax;
+    if (clip_mode == CONVROT_CLIP_MSE) {
+        WeightPass errs;
+        errs.given_amax = g_amax;
+        errs.row_err_out = row_err;
+        dispatch_weight(log2b, W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st, errs);
+        convrot::err_argmin_kernel<<<1, 64, 0, st>>>(row_err, N, g_alpha);
+        quant.given_alpha = g_alpha;
+    }
+    dispatch_weight(log2b, W, w_dtype, N, K, bits, clip_mode, Wq, w_scale, st, quant);
+    return launch_status("weight_rotate_quant (tensor-wise)");
 }
 
 convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, int block, int bits, void *Xq,

@@ -433,11 +433,22 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
 // ---------------------------------------------------------------------------
 constexpr int kMseGrid = 51;
 
+//
+// Tensor-wise scales use the same kernel in three passes (all optional
+// pointers null = the row-wise converter):
+//   row_amax_out   stats pass: write each row's absmax and stop;
+//   row_err_out    error pass: with the tensor's absmax `given_amax`, write each
+//                  row's float64 error for every grid point and stop;
+//   given_amax / given_alpha   quantize every row with that absmax and grid point.
 template <int LOG2B>
 __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *__restrict__ W, int dtype,
                                                                    int64_t N, int K, int rows, int bits,
                                                                    int clip_mode, void *__restrict__ Wq,
-                                                                   float *__restrict__ w_scale) {
+                                                                   float *__restrict__ w_scale,
+                                                                   const float *__restrict__ given_amax,
+                                                                   const int *__restrict__ given_alpha,
+                                                                   float *__restrict__ row_amax_out,
+                                                                   double *__restrict__ row_err_out) {
     __shared__ unsigned int s_amax[kMaxRowsPerCta];
     __shared__ float s_scale[kMaxRowsPerCta][kMseGrid];
     __shared__ double s_part[256];  // one partial sum per (row, segment of G lanes): at most 1024 / 4
@@ -486,12 +497,20 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
     for (int m = 1; m < G; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
     if (r < rows && (l & (G - 1)) == 0) atomicMax(&s_amax[r], __float_as_uint(amax));
     __syncthreads();
-    const int n_alpha = clip_mode == 1 ? kMseGrid : 1;
+    if (row_amax_out != nullptr) {  // stats pass (uniform across the block)
+        if (active && l == 0) row_amax_out[row] = __uint_as_float(s_amax[r]);
+        return;
+    }
+    const bool search = clip_mode == 1 && given_alpha == nullptr;
+    const int n_alpha = search ? kMseGrid : 1;
+    const int alpha0 = given_alpha != nullptr ? *given_alpha : 0;
     // grid point i: alpha = fp32((100 - i) / 100), s = fp32(fp32(alpha * amax) / qmax)
     if (r < rows) {
+        const float am = given_amax != nullptr ? *given_amax : __uint_as_float(s_amax[r]);
         for (int i = l; i < n_alpha; i += L) {
-            const float alpha = __fdiv_rn(static_cast<float>(100 - i), 100.0f);
-            s_scale[r][i] = __fdiv_rn(__fmul_rn(alpha, __uint_as_float(s_amax[r])), static_cast<float>(qmax));
+            const int ai = search ? i : alpha0;
+            const float alpha = __fdiv_rn(static_cast<float>(100 - ai), 100.0f);
+            s_scale[r][i] = __fdiv_rn(__fmul_rn(alpha, am), static_cast<float>(qmax));
         }
     }
     __syncthreads();
@@ -520,6 +539,7 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
             if (r < rows && l == 0) {
                 double tot = 0.0;
                 for (int sgi = 0; sgi < segs; ++sgi) tot += s_part[r * segs + sgi];
+                if (row_err_out != nullptr && active) row_err_out[row * kMseGrid + i] = tot;
                 if (tot < s_best_err[r]) {
                     s_best_err[r] = tot;
                     s_best[r] = i;
@@ -528,7 +548,7 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
             __syncthreads();
         }
     }
-    if (!active) return;
+    if (row_err_out != nullptr || !active) return;  // the error pass ends here
     const float s = s_scale[r][s_best[r]];
     const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
     if (l == 0) w_scale[row] = s;
@@ -546,6 +566,44 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
     }
     if (bits == 8) store_codes<8>(static_cast<int8_t *>(Wq) + row * K, elem0, q);
     else store_codes<4>(static_cast<uint8_t *>(Wq) + row * (K / 2), elem0, q);
+}
+
+
+// Tensor-wise pass helpers (one block each; offline).
+// The tensor's absmax: max over the rows' absmax values (order-free).
+__global__ void __launch_bounds__(1024) amax_reduce_kernel(const float *__restrict__ row_amax, int64_t N,
+                                                           float *__restrict__ out) {
+    __shared__ float s_max[32];
+    float m = 0.0f;
+    for (int64_t i = threadIdx.x; i < N; i += blockDim.x) m = fmaxf(m, row_amax[i]);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.0f;
+        for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t = fmaxf(t, s_max[w]);
+        *out = t;
+    }
+}
+
+// The clip choice: for every grid point the rows' float64 errors summed in row
+// order (thread i owns grid point i), then the first strict minimum.
+__global__ void __launch_bounds__(64) err_argmin_kernel(const double *__restrict__ row_err, int64_t N,
+                                                        int *__restrict__ alpha_out) {
+    __shared__ double s_tot[64];
+    const int i = threadIdx.x;
+    if (i < kMseGrid) {
+        double t = 0.0;
+        for (int64_t n = 0; n < N; ++n) t += row_err[n * kMseGrid + i];
+        s_tot[i] = t;
+    }
+    __syncthreads();
+    if (i == 0) {
+        int best = 0;
+        for (int j = 1; j < kMseGrid; ++j)
+            if (s_tot[j] < s_tot[best]) best = j;
+        *alpha_out = best;
+    }
 }
 
 

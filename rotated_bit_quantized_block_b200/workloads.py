@@ -22,6 +22,7 @@ class Linear:
     name: str
     K: int  # in-features (reduction dimension)
     N: int  # out-features
+    bits: int = 0  # 8 or 4 for this linear; 0 = the workload's width
 
 
 @dataclass(frozen=True)
@@ -36,6 +37,10 @@ class Workload:
     w_sigma: float
     seed: int
     description: str = field(default="", compare=False)
+
+    def bits_of(self, lin: Linear) -> int:
+        """Code width of one linear (per-layer choice, else the workload's)."""
+        return lin.bits or self.bits
 
     def ops(self) -> int:
         """Integer multiply-adds x2 of one pass over every linear."""
@@ -55,6 +60,11 @@ WORKLOADS = {
                            "ViT-L encoder linears, W4A4"),
     "dit_w8a8": Workload("dit_w8a8", 8192, DIT_LINEARS, 8, 128, 0.005, 50.0, 0.015, 3,
                          "DiT linears, batch 2 x 4096 tokens"),
+    # per-layer code width: attention linears W8A8, MLP linears W4A4
+    "vit_l_mixed": Workload("vit_l_mixed", 5184,
+                            (Linear("qkv", 1024, 3072, 8), Linear("proj", 1024, 1024, 8),
+                             Linear("fc1", 1024, 4096, 4), Linear("fc2", 4096, 1024, 4)),
+                            8, 128, 0.01, 30.0, 0.02, 5, "ViT-L encoder linears, W8A8 attention, W4A4 MLP"),
 }
 MSWEEP_M = (1, 16, 128, 1024, 4096, 16384)
 

@@ -123,3 +123,16 @@ def test_linear_workspace_bytes_adds_split_k_room(lib):
     assert lws(16384, 4096, 4096, 8) == ws(16384, 4096, 8) + 2048
     assert lws(-1, 4096, 4096, 8) == 0
     assert lws(4, 4096, 4096, 5) == 0
+
+
+def test_tensorwise_workspace_and_validation(lib):
+    ws = lib.convrot_tensorwise_workspace_bytes
+    assert ws(1000, 0) == 4096 + 256
+    assert ws(1000, 1) == 4096 + 256 + ((1000 * 51 * 8 + 255) // 256) * 256
+    assert ws(-1, 0) == 0 and ws(10, 7) == 0
+    q = lib.convrot_quantize_weight_tensorwise
+    assert q(None, 0, 0, 128, 64, 8, 1, None, None, None, 0, None) == binding.OK  # no rows: no-op
+    assert q(A16, 0, 64, 256, 64, 8, 1, A16, A16, A16, 100, None) == binding.ERR_WORKSPACE
+    assert q(A16, 0, 64, 256, 64, 8, 1, A16, A16, MIS, 1 << 20, None) == binding.ERR_ALIGNMENT
+    assert q(A16, 0, 64, 256, 64, 8, 3, A16, A16, A16, 1 << 20, None) == binding.ERR_INVALID_ARG
+    assert q(A16, 0, 64, 100, 64, 8, 0, A16, A16, A16, 1 << 20, None) == binding.ERR_INVALID_ARG

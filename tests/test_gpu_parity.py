@@ -252,11 +252,12 @@ def test_gemm_full_size_sampled_rows(bits):
 
 def linear_pair(w, idx, M=None, with_bias=False, sample=None):
     X, W, bias = wl.linear_inputs(w, idx, M=M, with_bias=with_bias)
-    lin = cr.QuantizedLinear(dev(W), None if bias is None else dev(bias), w.block, w.bits, cr.CLIP_MSE)
+    bits = w.bits_of(w.linears[idx])
+    lin = cr.QuantizedLinear(dev(W), None if bias is None else dev(bias), w.block, bits, cr.CLIP_MSE)
     y = host(lin(dev(X)))
-    qw, sw, _ = oracle.quantize_weight(W, w.block, w.bits, oracle.CLIP_MSE)
+    qw, sw, _ = oracle.quantize_weight(W, w.block, bits, oracle.CLIP_MSE)
     rows = np.arange(X.shape[0]) if sample is None else sample
-    yr = oracle.linear(X[rows], qw, sw, w.block, w.bits, bias)
+    yr = oracle.linear(X[rows], qw, sw, w.block, bits, bias)
     ref = X[rows].astype(np.float64) @ W.astype(np.float64).T
     if bias is not None:
         ref += bias.astype(np.float64)
@@ -280,6 +281,16 @@ def test_linear_vit_full_size_sampled(name, idx):
     y, yr, ref = linear_pair(w, idx, sample=rows)
     assert rel_fro(y, yr) <= REL_FRO
     assert rel_fro(y, ref) <= (0.02 if w.bits == 8 else 0.3)
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2, 3])
+def test_linear_mixed_widths_full_size_sampled(idx):
+    """Per-layer code width (W8A8 attention, W4A4 MLP) at the ViT-L size."""
+    w = wl.WORKLOADS["vit_l_mixed"]
+    rows = np.unique(np.concatenate([[0, w.M - 1], np.linspace(0, w.M - 1, 32).astype(int)]))
+    y, yr, ref = linear_pair(w, idx, sample=rows)
+    assert rel_fro(y, yr) <= REL_FRO
+    assert rel_fro(y, ref) <= (0.02 if w.bits_of(w.linears[idx]) == 8 else 0.3)
 
 
 @pytest.mark.parametrize("idx", [0, 1, 2])
@@ -387,3 +398,43 @@ def test_linear_pair_tiles_bit_exact_sampled(bits):
     rows = pair_rows(M)
     yr = oracle.gemm_dequant(qx[rows], sx[rows], unpack(host(Wq), bits), host(sw), bias)
     assert np.array_equal(y[rows].view(np.uint16), yr.view(np.uint16))
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("clip", [0, 1])
+@pytest.mark.parametrize("N,K,b", [(300, 1024, 128), (64, 4096, 256), (7, 256, 64)])
+def test_weight_tensorwise_matches_oracle(N, K, b, bits, clip):
+    """One scale for the tensor: the clip choice is the oracle's (or a near-tie
+    under the oracle's own errors), the scale agrees, the codes meet the code bar."""
+    W = wl.weight(N, K, 0.02, seed=N + K + bits)
+    W[N // 2, ::17] *= 40  # a few large weights, so that clipping matters
+    Wq, sw = cr.convrot_quantize_weight_tensorwise(dev(W), b, bits, clip)
+    sw = host(sw)
+    codes = unpack(host(Wq), bits)
+    rc, rs, ra, rerr = oracle.quantize_weight_tensorwise(W, b, bits, clip, want_errs=True)
+    assert np.all(sw == sw[0])
+    # the oracle's tensor absmax (rotation in float64, rounded to fp32)
+    amax_o = float(np.max(np.abs(oracle.rotate(W.astype(np.float64), b)[1])))
+    s_gpu = float(sw[0])
+    # the GPU's scale is a grid point of (nearly) the same absmax ...
+    cand = [i for i in (range(oracle.MSE_GRID) if clip == 1 else [0])
+            if abs(float(oracle.scale(amax_o, oracle.alpha(i), bits)) - s_gpu) <= 2e-6 * s_gpu]
+    assert cand, "the GPU's scale is not a grid point of the tensor's absmax"
+    # ... whose total error is the oracle's minimum or a near-tie with it
+    if clip == 1:
+        assert min(rerr[i] for i in cand) <= rerr[ra] * (1 + 1e-6)
+    if abs(s_gpu - float(rs[0])) <= 2e-6 * float(rs[0]):
+        assert_codes_close(codes, rc)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_linear_with_tensorwise_weights(bits):
+    """The linears consume tensor-wise scales unchanged."""
+    w = wl.WORKLOADS["vit_l_w8a8"]
+    X, W, bias = wl.linear_inputs(w, 0, M=300, with_bias=True)
+    Wq, sw = cr.convrot_quantize_weight_tensorwise(dev(W), 128, bits, cr.CLIP_MSE)
+    fn = cr.convrot_linear_w8a8 if bits == 8 else cr.convrot_linear_w4a4
+    y = host(fn(dev(X), Wq, sw, 128, bias=dev(bias)))
+    qw, swr, _ = oracle.quantize_weight_tensorwise(W, 128, bits, oracle.CLIP_MSE)
+    yr = oracle.linear(X, qw, swr, 128, bits, bias)
+    assert rel_fro(y, yr) <= REL_FRO
