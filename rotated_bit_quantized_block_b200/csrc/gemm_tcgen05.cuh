@@ -70,11 +70,14 @@ struct GemmCfg {
     static constexpr int CONV_ROWS = (A4 ? BM : 0) + (B4 ? B_ROWS : 0);  // rows widened per stage
     // arrivals completing an MMA stage: the producer (TMA bytes) and/or the four
     // converter warps (of both CTAs of a pair)
-    static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + (W4 ? 4 * CTAS : 0);
+    // converter warps widening int4 (token-major: 8, so that widening keeps pace with the MMA)
+    static constexpr int CONV_WARPS = !W4 ? 0 : (SWAP ? 4 : 8);
+    static constexpr int CONV_THREADS = 32 * CONV_WARPS;
+    static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + CONV_WARPS * CTAS;
     static constexpr int TMEM_COLS = 2 * BN;
     // epilogue warps: per TMEM lane quarter, EPI_WARPS / 4 warps split the columns
     // (token-major: four, so that enough warps hide the dequant's latencies)
-    static constexpr int EPI_WARPS = SWAP ? 8 : 16;
+    static constexpr int EPI_WARPS = (SWAP || W4) ? 8 : 16;
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // accumulator columns per epilogue warp
     // token-major: 32-column chunks (one TMEM load, one 32 x 32 fp16 output box);
     // feature-major: 16- or 32-column TMEM loads, stored directly
@@ -83,7 +86,7 @@ struct GemmCfg {
     static constexpr int OUT_BYTES = SWAP ? 0 : EPI_WARPS * OUT_BOX_BYTES;
     static constexpr int SCALE_BYTES = BN * 4 + BN * 2;  // the tile's column scale (fp32) and bias (fp16)
     static constexpr int FIRST_CONV_WARP = 2 + EPI_WARPS;
-    static constexpr int NUM_THREADS = 32 * (FIRST_CONV_WARP + (W4 ? 4 : 0));
+    static constexpr int NUM_THREADS = 32 * (FIRST_CONV_WARP + CONV_WARPS);
     static constexpr int FIXED_BARRIERS = 2 * PSTAGES + 4 + 1 + 2 + 2;
     // MMA ring depth: as many stages as fit in the shared-memory budget (at most 12)
     static constexpr int SMEM_LIMIT = 232448;
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         }
         for (int i = 0; i < PSTAGES; ++i) {
             mbar_init(&pfull[i], 1);
-            mbar_init(&pempty[i], 128);
+            mbar_init(&pempty[i], Cfg::CONV_THREADS);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tmem_full[i], 1);
@@ -569,7 +572,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         if (!Cfg::SWAP && lane == 0) bulk_wait_group_all();
     } else if (Cfg::W4) {
         // ------------------------------------------------------------ int4 -> int8 converters
-        const int ct = threadIdx.x - 32 * Cfg::FIRST_CONV_WARP;  // 0..127
+        const int ct = threadIdx.x - 32 * Cfg::FIRST_CONV_WARP;  // 0 .. CONV_THREADS-1
         int ps = 0, us = 0;
         uint32_t pph = 0, uph = 0;
         bool ok = true;
@@ -584,7 +587,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                 uint8_t *dst = ring + us * Cfg::STAGE_BYTES + (Cfg::A4 ? 0 : Cfg::A_BYTES);
                 constexpr int PIECES = Cfg::CONV_ROWS * (Cfg::BK / 16);  // 16 codes per piece
 #pragma unroll 4
-                for (int idx = ct; idx < PIECES; idx += 128) {
+                for (int idx = ct; idx < PIECES; idx += Cfg::CONV_THREADS) {
                     const int rr = idx >> 3, piece = idx & 7;  // widened row; 16-byte chunk in the row
                     const uint2 p = *reinterpret_cast<const uint2 *>(src + rr * 64 + piece * 8);
                     *reinterpret_cast<uint4 *>(dst + rr * 128 + ((piece ^ (rr & 7)) << 4)) = widen_int4x16(p);
