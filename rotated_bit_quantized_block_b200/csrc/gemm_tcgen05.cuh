@@ -71,7 +71,7 @@ struct GemmCfg {
     // arrivals completing an MMA stage: the producer (TMA bytes) and/or the four
     // converter warps (of both CTAs of a pair)
     // converter warps widening int4 (token-major: 8, so that widening keeps pace with the MMA)
-    static constexpr int CONV_WARPS = !W4 ? 0 : (SWAP ? 4 : 8);
+    static constexpr int CONV_WARPS = !W4 ? 0 : (SWAP ? 4 : 12);
     static constexpr int CONV_THREADS = 32 * CONV_WARPS;
     static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + CONV_WARPS * CTAS;
     static constexpr int TMEM_COLS = 2 * BN;
