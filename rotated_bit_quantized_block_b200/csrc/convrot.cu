@@ -331,7 +331,7 @@ constexpr int64_t kMaxSplitFeatures = 32768;     // split K only for N up to thi
 // narrowed to 128 when 256-wide tiles would leave more than half the SMs idle.
 // (Measured on B200 with CUDA-graph launches: feature-major wins up to 128
 // tokens, token-major from 192.)
-GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split) {
+GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split, bool w4 = false) {
     GemmPlan p;
     if (M <= kSwapMaxTokens) {
         p.swap = true;
@@ -345,14 +345,30 @@ GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split) {
         }
         return p;
     }
+    // tile width: fewest rounds of tiles weighted by a tile's measured relative
+    // cost (B200, CUDA-graph-timed: a 192-wide tile takes 0.83 of a 256-wide
+    // one's time with int8 weights, 0.80 with widened int4; a 128-wide one
+    // 0.78 / 0.63), ties to the wider tile
     const int64_t tiles_m = (M + 127) / 128;
-    const int64_t tiles_256 = tiles_m * ((N + 255) / 256);
-    p.bn = (N >= 256 && 2 * tiles_256 > sms) ? 256 : 128;
-    p.tiles = tiles_m * ((N + p.bn - 1) / p.bn);
+    const int widths[3] = {256, 192, 128};
+    const double cost8[3] = {1.0, 0.83, 0.78}, cost4[3] = {1.0, 0.80, 0.63};
+    double best = -1.0;
+    for (int i = 0; i < 3; ++i) {
+        const int bn = widths[i];
+        if (bn > 128 && N < bn) continue;
+        const int64_t tiles = tiles_m * ((N + bn - 1) / bn);
+        const double c = static_cast<double>((tiles + sms - 1) / sms) * (w4 ? cost4[i] : cost8[i]);
+        if (best < 0.0 || c < best - 1e-9) {
+            best = c;
+            p.bn = bn;
+            p.tiles = tiles;
+        }
+    }
     // CTA pairs halve each SM's operand traffic, which pays where the main loop
-    // dominates: deep K and at least two rounds of 256 x 256 tiles
+    // dominates: deep K and at least two rounds of 256 x 256 tiles (int8
+    // weights; with widened int4 weights pairs measured slower)
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    p.pair = p.bn == 256 && K >= 1536 && pair_tiles >= sms;
+    p.pair = p.bn == 256 && !w4 && K >= 1536 && pair_tiles >= sms;
     return p;
 }
 
@@ -443,11 +459,15 @@ convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const vo
     if (p.swap)
         return launch_gemm_cfg<GemmCfg<kSwapTokens, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y,
                                                                    acc_out, st, p.splits, acc_buf, counters);
+    if (p.bn == 192)
+        return launch_gemm_cfg<GemmCfg<192, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
+                                                     nullptr, nullptr);
     if (p.bn == 256) {
-        if constexpr (!X4) {
+        if constexpr (!X4 && !W4) {
             if (p.pair)
-                return launch_gemm_cfg<GemmCfg<256, false, W4, false, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias,
-                                                                             Y, acc_out, st, 1, nullptr, nullptr);
+                return launch_gemm_cfg<GemmCfg<256, false, false, false, true>>(info, dev, Xc, Wc, M, N, K, sx, sw,
+                                                                                bias, Y, acc_out, st, 1, nullptr,
+                                                                                nullptr);
         }
         return launch_gemm_cfg<GemmCfg<256, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
                                                      nullptr, nullptr);
@@ -689,7 +709,7 @@ static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace
     CR_TRY(current_device(&dev, &info));
     // split K only when the workspace holds the counters and the sum buffer
     // (which the activation half zeroed)
-    GemmPlan p = plan_gemm(info->sms, M, N, K, true);
+    GemmPlan p = plan_gemm(info->sms, M, N, K, true, bits == 4);
     const size_t base = convrot_workspace_bytes(M, K, bits) + kCounterBytes;
     if (p.splits > 1 && workspace_bytes < base + split_buffer_bytes(p, M, N)) p.splits = 1;
     if (bits == 8)
@@ -753,7 +773,7 @@ static convrot_status_t gemm_impl(bool w4, const void *Xq, const float *x_scale,
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const GemmPlan p = plan_gemm(info->sms, M, N, K, false);  // no workspace: no split-K
+    const GemmPlan p = plan_gemm(info->sms, M, N, K, false, w4);  // no workspace: no split-K
     if (w4) return launch_gemm<true, true>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st, p);
     return launch_gemm<false, false>(info, dev, Xq, Wq, M, N, K, x_scale, w_scale, bias, Y, acc_out, st, p);
 }

@@ -74,10 +74,11 @@ struct GemmCfg {
     static constexpr int CONV_WARPS = !W4 ? 0 : (SWAP ? 4 : 12);
     static constexpr int CONV_THREADS = 32 * CONV_WARPS;
     static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + CONV_WARPS * CTAS;
-    static constexpr int TMEM_COLS = 2 * BN;
+    // two accumulators; the allocation is a power of two of at least 32 columns
+    static constexpr int TMEM_COLS = 2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512));
     // epilogue warps: per TMEM lane quarter, EPI_WARPS / 4 warps split the columns
     // (token-major: four, so that enough warps hide the dequant's latencies)
-    static constexpr int EPI_WARPS = (SWAP || W4) ? 8 : 16;
+    static constexpr int EPI_WARPS = (SWAP || W4 || BN % 128 != 0) ? 8 : 16;
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // accumulator columns per epilogue warp
     // token-major: 32-column chunks (one TMEM load, one 32 x 32 fp16 output box);
     // feature-major: 16- or 32-column TMEM loads, stored directly
@@ -99,10 +100,11 @@ struct GemmCfg {
                                       OUT_BYTES + SCALE_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t IDESC = idesc_i8(TILE_M, BN);
     static_assert(STAGES >= 2, "pipeline depth");
-    static_assert(!PAIR || (!SWAP && !A4 && BN == 256), "CTA pairs: token-major, int8 A, 256-wide tiles");
+    static_assert(!PAIR || (!SWAP && !A4 && !B4 && BN == 256), "CTA pairs: token-major W8A8, 256-wide tiles");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(SWAP ? (BN == 32 || BN == 64 || BN == 128 || BN == 256) : (BN % 64 == 0 && BN >= 64 && BN <= 256),
                   "tile width");
+    static_assert(TMEM_COLS >= 2 * BN, "accumulators fit the allocation");
     static_assert(EPI_COLS % CHUNK == 0, "epilogue chunking");
 };
 

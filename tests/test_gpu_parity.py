@@ -381,8 +381,9 @@ def test_gemm_pair_tiles_bit_exact_sampled(M, N, K):
 
 @pytest.mark.parametrize("bits", [8, 4])
 def test_linear_pair_tiles_bit_exact_sampled(bits):
-    """The linear on CTA pairs (int8 activations, int8 or widened int4 weights):
-    the output equals the oracle's GEMM of the workspace's codes on sampled rows."""
+    """The linear at a shape the plan runs on CTA pairs for int8 weights (and on
+    single-CTA 256-wide tiles for int4): the output equals the oracle's GEMM of
+    the workspace's codes on sampled rows."""
     M, N, K = 2700, 4000, 1536
     X = wl.activations(M, K, 0.01, 30.0, seed=17)
     W = wl.weight(N, K, 0.02, seed=18)
