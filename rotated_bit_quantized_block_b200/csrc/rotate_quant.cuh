@@ -432,6 +432,7 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
 // (lanes, then row segments in index order), so the choice is deterministic.
 // ---------------------------------------------------------------------------
 constexpr int kMseGrid = 51;
+constexpr int kMseBatch = 4;  // grid points scored per pass (one pair of block barriers per pass)
 
 //
 // Tensor-wise scales use the same kernel in three passes (all optional
@@ -451,7 +452,8 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
                                                                    double *__restrict__ row_err_out) {
     __shared__ unsigned int s_amax[kMaxRowsPerCta];
     __shared__ float s_scale[kMaxRowsPerCta][kMseGrid];
-    __shared__ double s_part[256];  // one partial sum per (row, segment of G lanes): at most 1024 / 4
+    // one partial sum per (row, segment of G lanes, grid point of the batch): at most 1024 / 4 x batch
+    __shared__ double s_part[256 * kMseBatch];
     __shared__ double s_best_err[kMaxRowsPerCta];
     __shared__ int s_best[kMaxRowsPerCta];
     const int L = K / kElemsPerThread;
@@ -515,11 +517,18 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
     }
     __syncthreads();
     if (n_alpha > 1) {
-        for (int i = 0; i < n_alpha; ++i) {
-            const float s = r < rows ? s_scale[r][i] : 0.0f;
-            const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
-            const double sd = static_cast<double>(s);
-            double err = 0.0;
+        // kMseBatch grid points per pass; each point's float64 error is summed in
+        // the same order as one point at a time (elements, lanes, then segments)
+        for (int i0 = 0; i0 < n_alpha; i0 += kMseBatch) {
+            float inv[kMseBatch];
+            double sd[kMseBatch], err[kMseBatch];
+#pragma unroll
+            for (int a = 0; a < kMseBatch; ++a) {
+                const float s = (r < rows && i0 + a < n_alpha) ? s_scale[r][i0 + a] : 0.0f;
+                inv[a] = s == 0.0f ? 0.0f : __frcp_rn(s);
+                sd[a] = static_cast<double>(s);
+                err[a] = 0.0;
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -527,22 +536,32 @@ __global__ void __launch_bounds__(1024) weight_rotate_quant_kernel(const void *_
                     const float xs[2] = {v[h][e].x, v[h][e].y};
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
-                        const float q = quant_clamped(xs[c], inv, qmin, qmax);
-                        const double d = fma(-sd, static_cast<double>(q), static_cast<double>(xs[c]));
-                        err = fma(d, d, err);
+#pragma unroll
+                        for (int a = 0; a < kMseBatch; ++a) {
+                            const float q = quant_clamped(xs[c], inv[a], qmin, qmax);
+                            const double d = fma(-sd[a], static_cast<double>(q), static_cast<double>(xs[c]));
+                            err[a] = fma(d, d, err[a]);
+                        }
                     }
                 }
             }
-            for (int m = 1; m < G; m <<= 1) err += __shfl_xor_sync(0xffffffffu, err, m);
-            if (r < rows && (l & (G - 1)) == 0) s_part[r * segs + l / G] = err;
+#pragma unroll
+            for (int a = 0; a < kMseBatch; ++a)
+                for (int m = 1; m < G; m <<= 1) err[a] += __shfl_xor_sync(0xffffffffu, err[a], m);
+            if (r < rows && (l & (G - 1)) == 0) {
+#pragma unroll
+                for (int a = 0; a < kMseBatch; ++a) s_part[(r * segs + l / G) * kMseBatch + a] = err[a];
+            }
             __syncthreads();
             if (r < rows && l == 0) {
-                double tot = 0.0;
-                for (int sgi = 0; sgi < segs; ++sgi) tot += s_part[r * segs + sgi];
-                if (row_err_out != nullptr && active) row_err_out[row * kMseGrid + i] = tot;
-                if (tot < s_best_err[r]) {
-                    s_best_err[r] = tot;
-                    s_best[r] = i;
+                for (int a = 0; a < kMseBatch && i0 + a < n_alpha; ++a) {
+                    double tot = 0.0;
+                    for (int sgi = 0; sgi < segs; ++sgi) tot += s_part[(r * segs + sgi) * kMseBatch + a];
+                    if (row_err_out != nullptr && active) row_err_out[row * kMseGrid + i0 + a] = tot;
+                    if (tot < s_best_err[r]) {
+                        s_best_err[r] = tot;
+                        s_best[r] = i0 + a;
+                    }
                 }
             }
             __syncthreads();
