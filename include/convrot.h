@@ -133,8 +133,10 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
 
 /*
  * Workspace size that also lets the linear split the K loop of its GEMM across
- * SMs.  For few tokens (M <= 128) the GEMM runs feature-major (128 output
- * features x 32 tokens per tile) and has too few tiles to fill the GPU; with this
+ * SMs.  For the fewest tokens (M <= 4 with int8 weights, M <= 8 with int4) the
+ * GEMM is a weight-streaming kernel that needs no split.  Up to M = 128 it
+ * runs feature-major (128 output features x 32 tokens per tile) and has too
+ * few tiles to fill the GPU; with this
  * workspace the K slices of a tile run on separate SMs and add their int32
  * partials into an M x N buffer.  Size: convrot_workspace_bytes(M, K, bits)
  * plus 2 KB of split-K counters plus that buffer (rounded up to 256 bytes)

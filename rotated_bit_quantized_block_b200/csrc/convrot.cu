@@ -13,6 +13,7 @@
 #include "../../include/convrot.h"
 #include "device_utils.cuh"
 #include "gemm_tcgen05.cuh"
+#include "gemv.cuh"
 #include "rotate_quant.cuh"
 
 namespace {
@@ -313,6 +314,7 @@ convrot_status_t rotate_quant_act_impl(const void *X, int64_t M, int64_t K, int 
 struct GemmPlan {
     bool swap = false;  // feature-major (weights on the MMA's 128-row side)
     bool pair = false;  // token-major 256 x 256 tiles on CTA pairs (cta_group::2)
+    bool gemv = false;  // at most 16 tokens with int8 activation codes: weight-streaming kernel
     int bn = 256;       // MMA N: output features (token-major) or tokens (feature-major)
     int splits = 1;
     int64_t tiles = 0;
@@ -337,7 +339,12 @@ GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split, b
         p.swap = true;
         p.bn = kSwapTokens;
         p.tiles = ((N + 127) / 128) * ((M + p.bn - 1) / p.bn);
-        if (allow_split && p.tiles > 0 && p.tiles <= kMaxSplitTiles && N <= kMaxSplitFeatures) {
+        // for the fewest tokens the weight-streaming kernel runs instead (int8
+        // activation codes; the feature-major tiles stay for packed ones).
+        // Measured on B200 (K = N = 4096, CUDA graphs): faster up to 4 tokens
+        // with int8 weights (4.9 against 8.2 us at M = 1), up to 8 with int4
+        p.gemv = M <= (w4 ? 8 : 4);
+        if (allow_split && !p.gemv && p.tiles > 0 && p.tiles <= kMaxSplitTiles && N <= kMaxSplitFeatures) {
             int64_t s = sms / p.tiles;
             if (s > 8) s = 8;
             if (s > K / 1024) s = K / 1024;
@@ -449,6 +456,31 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, cons
     return launch_status("gemm_i8_tcgen05");
 }
 
+// Weight-streaming GEMM for M <= 16 tokens (int8 activation codes; W4 = packed
+// int4 weights): blocks of 4 output features, warps splitting K.
+template <bool W4, int MT>
+convrot_status_t launch_gemv_mt(const void *Xc, const void *Wc, int64_t M, int64_t N, int64_t K, const float *sx,
+                                const float *sw, const void *bias, void *Y, int32_t *acc_out, cudaStream_t st) {
+    int64_t nw = K / convrot::kGemvChunk;
+    nw = nw < 1 ? 1 : (nw > 8 ? 8 : nw);
+    const int64_t grid = (N + convrot::kGemvFeatures - 1) / convrot::kGemvFeatures;
+    launch_pdl(convrot::gemv_i8_kernel<W4, MT>, dim3(static_cast<unsigned>(grid)), dim3(static_cast<unsigned>(32 * nw)),
+               0, st, static_cast<const int8_t *>(Xc), sx, static_cast<const uint8_t *>(Wc), sw,
+               static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out, static_cast<int>(M),
+               static_cast<int>(N), static_cast<int>(K));
+    return launch_status("gemv_i8");
+}
+
+template <bool W4>
+convrot_status_t launch_gemv(const void *Xc, const void *Wc, int64_t M, int64_t N, int64_t K, const float *sx,
+                             const float *sw, const void *bias, void *Y, int32_t *acc_out, cudaStream_t st) {
+    if (M <= 1) return launch_gemv_mt<W4, 1>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
+    if (M <= 2) return launch_gemv_mt<W4, 2>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
+    if (M <= 4) return launch_gemv_mt<W4, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
+    if (M <= 8) return launch_gemv_mt<W4, 8>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
+    return launch_gemv_mt<W4, 16>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
+}
+
 // X4 / W4: activation / weight codes packed int4.
 template <bool X4, bool W4>
 convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const void *Wc, int64_t M, int64_t N,
@@ -456,6 +488,9 @@ convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const vo
                              int32_t *acc_out, cudaStream_t st, const GemmPlan &p, int32_t *acc_buf = nullptr,
                              unsigned int *counters = nullptr) {
     using convrot::GemmCfg;
+    if constexpr (!X4) {
+        if (p.gemv) return launch_gemv<W4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
+    }
     if (p.swap)
         return launch_gemm_cfg<GemmCfg<kSwapTokens, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y,
                                                                    acc_out, st, p.splits, acc_buf, counters);
@@ -536,7 +571,7 @@ size_t convrot_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits)
         cudaGetLastError();
     }
     if (M == 0 || N == 0 || K % 128 != 0 || K < 128) return base + kCounterBytes;
-    return base + kCounterBytes + split_buffer_bytes(plan_gemm(sms, M, N, K, true), M, N);
+    return base + kCounterBytes + split_buffer_bytes(plan_gemm(sms, M, N, K, true, bits == 4), M, N);
 }
 
 convrot_status_t convrot_quantize_weight(const void *W, int w_dtype, int64_t N, int64_t K, int block, int bits,
@@ -682,7 +717,7 @@ static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int
     if (workspace_bytes > base) {
         size_t cap;
         if (n_features >= 0) {
-            const GemmPlan p = plan_gemm(info->sms, M, n_features, K, true);
+            const GemmPlan p = plan_gemm(info->sms, M, n_features, K, true, bits == 4);
             cap = kCounterBytes + split_buffer_bytes(p, M, n_features);
         } else {
             cap = kCounterBytes + (M <= kSwapMaxTokens ? round256(static_cast<size_t>(M) * kMaxSplitFeatures * 4) : 0);

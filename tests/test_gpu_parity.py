@@ -439,3 +439,23 @@ def test_linear_with_tensorwise_weights(bits):
     qw, swr, _ = oracle.quantize_weight_tensorwise(W, 128, bits, oracle.CLIP_MSE)
     yr = oracle.linear(X, qw, swr, 128, bits, bias)
     assert rel_fro(y, yr) <= REL_FRO
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (3, 1000, 1024), (4, 2056, 640), (8, 3072, 128), (7, 520, 8192)])
+def test_weight_streaming_gemm_bit_exact(M, N, K, bits):
+    """For the fewest tokens the linear's GEMM streams the weights (dp4a, exact
+    int32): bit-exact against the oracle's GEMM of the workspace's codes, ragged N."""
+    X = wl.activations(M, K, 0.01, 30.0, seed=M + K)
+    W = wl.weight(N, K, 0.02, seed=N)
+    bias = wl.bias(N, seed=4)
+    Wq, sw = cr.convrot_quantize_weight(dev(W), 128, bits, cr.CLIP_MSE)
+    fn = cr.convrot_linear_w8a8 if bits == 8 else cr.convrot_linear_w4a4
+    ws = torch.empty(cr.convrot_linear_workspace_bytes(M, K, N, bits), dtype=torch.uint8, device="cuda")
+    y = host(fn(dev(X), Wq, sw, 128, bias=dev(bias), workspace=ws))
+    raw = host(ws)
+    qx = raw[: M * K].view(np.int8).reshape(M, K)
+    off = (M * K + 255) // 256 * 256
+    sx = raw[off: off + 4 * M].view(np.float32)
+    yr = oracle.gemm_dequant(qx, sx, unpack(host(Wq), bits), host(sw), bias)
+    assert np.array_equal(y.view(np.uint16), yr.view(np.uint16))
