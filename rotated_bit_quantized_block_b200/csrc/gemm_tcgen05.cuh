@@ -14,10 +14,10 @@
 // 128 x BN, K step 128 bytes.
 //   warp 0      TMA producer (one elected lane): A and B tiles -> smem ring
 //   warp 1      TMEM allocator + MMA issuer (one lane): 4 x tcgen05.mma per K step
-//   epilogue    16 warps (token-major) or 8 (feature-major): tcgen05.ld of
-//               the accumulator, scale, fp16, store
-//   converters  4 warps (int4 operands only): nibble -> byte widening between
-//               a packed ring and the MMA ring
+//   epilogue    16 warps (token-major, int8 weights, 128- or 256-wide tiles)
+//               or 8: tcgen05.ld of the accumulator, scale, fp16, store
+//   converters  int4 operands only, 12 warps (token-major) or 4: nibble ->
+//               byte widening between a packed ring and the MMA ring
 // Two TMEM accumulators (2 x BN columns) let the epilogue of one tile overlap
 // the main loop of the next.  No TMA multicast is used anywhere.
 //
@@ -66,14 +66,13 @@ struct GemmCfg {
     static constexpr int PA_BYTES = A4 ? A_BYTES / 2 : 0;
     static constexpr int PB_BYTES = B4 ? B_BYTES / 2 : 0;
     static constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
-    static constexpr int PSTAGES = !W4 ? 0 : (!SWAP && BN == 256 && !PAIR ? 3 : 4);
+    static constexpr int PSTAGES = !W4 ? 0 : (!SWAP && BN == 256 ? 3 : 4);
     static constexpr int CONV_ROWS = (A4 ? BM : 0) + (B4 ? B_ROWS : 0);  // rows widened per stage
-    // arrivals completing an MMA stage: the producer (TMA bytes) and/or the four
-    // converter warps (of both CTAs of a pair)
-    // converter warps widening int4 (token-major: 8, so that widening keeps pace with the MMA)
+    // converter warps widening int4 (token-major: 12, so that widening keeps pace with the MMA)
     static constexpr int CONV_WARPS = !W4 ? 0 : (SWAP ? 4 : 12);
     static constexpr int CONV_THREADS = 32 * CONV_WARPS;
-    static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + CONV_WARPS * CTAS;
+    // arrivals completing an MMA stage: the producer (TMA bytes) and/or one per converter warp
+    static constexpr int FULL_COUNT = (TMA_RING ? 1 : 0) + CONV_WARPS;
     // two accumulators; the allocation is a power of two of at least 32 columns
     static constexpr int TMEM_COLS = 2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512));
     // epilogue warps: per TMEM lane quarter, EPI_WARPS / 4 warps split the columns
@@ -286,14 +285,11 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                         uint8_t *dst = ring + s * Cfg::STAGE_BYTES;
                         if (Cfg::PAIR) {
                             // both CTAs' bytes land on the even CTA's barrier
-                            if (leader)
-                                mbar_arrive_expect_tx(&full[s],
-                                                      2 * (Cfg::A_BYTES + (Cfg::B4 ? 0 : Cfg::B_BYTES)));
+                            if (leader) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
                             const uint32_t bar = cluster_addr(&full[s], 0);
                             tma_load_2d_pair(dst, &tmA, bar, kb * Cfg::BK, tm * Cfg::TILE_M + rank * BM);
-                            if (!Cfg::B4)
-                                tma_load_2d_pair(dst + Cfg::A_BYTES, &tmB, bar, kb * Cfg::BK,
-                                                 tn * BN + rank * Cfg::B_ROWS);
+                            tma_load_2d_pair(dst + Cfg::A_BYTES, &tmB, bar, kb * Cfg::BK,
+                                             tn * BN + rank * Cfg::B_ROWS);
                         } else {
                             mbar_arrive_expect_tx(&full[s],
                                                   (Cfg::A4 ? 0 : Cfg::A_BYTES) + (Cfg::B4 ? 0 : Cfg::B_BYTES));
@@ -316,8 +312,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                         mbar_arrive_expect_tx(&pfull[ps], Cfg::PSTAGE_BYTES);
                         if (Cfg::A4) tma_load_2d(dst, &tmA, &pfull[ps], kb * (Cfg::BK / 2), tm * BM);
                         if (Cfg::B4)
-                            tma_load_2d(dst + Cfg::PA_BYTES, &tmB, &pfull[ps], kb * (Cfg::BK / 2),
-                                        tn * BN + rank * Cfg::B_ROWS);
+                            tma_load_2d(dst + Cfg::PA_BYTES, &tmB, &pfull[ps], kb * (Cfg::BK / 2), tn * BN);
                         pfilled[ps] = true;
                         plast_parity[ps] = pph;
                         if (++ps == PSTAGES) {
@@ -597,10 +592,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                 // the widened bytes are visible to the tensor core before the stage is signalled
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    if (Cfg::PAIR) mbar_arrive_cluster(cluster_addr(&full[us], 0));
-                    else mbar_arrive(&full[us]);
-                }
+                if (lane == 0) mbar_arrive(&full[us]);
                 mbar_arrive(&pempty[ps]);
                 if (++ps == PSTAGES) {
                     ps = 0;
