@@ -459,3 +459,31 @@ def test_weight_streaming_gemm_bit_exact(M, N, K, bits):
     sx = raw[off: off + 4 * M].view(np.float32)
     yr = oracle.gemm_dequant(qx, sx, unpack(host(Wq), bits), host(sw), bias)
     assert np.array_equal(y.view(np.uint16), yr.view(np.uint16))
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (3, 2056, 8192), (64, 1024, 4096), (700, 1024, 1024),
+                                   (2700, 4000, 1536)])
+def test_linear_reads_weights_written_just_before(M, N, K, bits):
+    """Both launches of the linear run with programmatic dependent launch.
+    Weights quantized by the kernel launched right before the linear, on the
+    same stream with no synchronization, must be the ones the GEMM reads: the
+    output equals that of the same linear run after a device sync (every
+    weight-streaming, feature-major split, token-major and CTA-pair plan)."""
+    X = wl.activations(M, K, 0.01, 30.0, seed=M + 11)
+    W = wl.weight(N, K, 0.02, seed=N + 11)
+    bias = wl.bias(N, seed=6)
+    Xd, Wd, bd = dev(X), dev(W), dev(bias)
+    shape = cr.code_shape(N, K, bits)
+    Wq = torch.zeros(shape, dtype=cr.code_dtype(bits), device="cuda")
+    sw = torch.zeros(N, dtype=torch.float32, device="cuda")
+    ws = torch.empty(cr.convrot_linear_workspace_bytes(M, K, N, bits), dtype=torch.uint8, device="cuda")
+    fn = cr.convrot_linear_w8a8 if bits == 8 else cr.convrot_linear_w4a4
+    torch.cuda.synchronize()
+    cr.convrot_quantize_weight(Wd, 128, bits, cr.CLIP_ABSMAX, Wq=Wq, w_scale=sw)
+    y_chained = host(fn(Xd, Wq, sw, 128, bias=bd, workspace=ws))
+    torch.cuda.synchronize()
+    y_after = host(fn(Xd, Wq, sw, 128, bias=bd, workspace=ws))
+    assert np.array_equal(y_chained.view(np.uint16), y_after.view(np.uint16))
+    # and the weights really changed: the zero codes give bias-only rows
+    assert not np.array_equal(y_after.view(np.uint16), np.broadcast_to(bias.astype(np.float16), y_after.shape).view(np.uint16))
