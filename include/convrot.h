@@ -138,12 +138,18 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
  * runs feature-major (128 output features x 32 tokens per tile) and has too
  * few tiles to fill the GPU; with this
  * workspace the K slices of a tile run on separate SMs and add their int32
- * partials into an M x N buffer.  Size: convrot_workspace_bytes(M, K, bits)
- * plus 2 KB of split-K counters plus that buffer (rounded up to 256 bytes)
- * when the GEMM will split.  The activation half of the linear zeroes what
- * follows the scales (the counters and the buffer); the GEMM half leaves both
- * zeroed again.  With only the minimum workspace the linears never split.
- * Depends on the current device's SM count.  Returns 0 for invalid arguments.
+ * partials into an M x N buffer.  For more tokens, where the 128 x 256 output
+ * tiles fill some but not all SMs in their last round (and CTA pairs are not
+ * used), the GEMM runs stream-K: every SM takes an equal share of all tiles'
+ * K steps, and a tile shared by two SMs is summed from one int32 partial tile
+ * (128 x 256) that the first of them stores in a slot of this workspace.
+ * Size: convrot_workspace_bytes(M, K, bits) plus 2 KB of split-K counters plus
+ * that buffer (rounded up to 256 bytes) or (SMs + 1) partial-tile slots of
+ * 128 KB.  The activation half of the linear zeroes the counters and the M x N
+ * buffer; the GEMM half leaves both zeroed again (the partial-tile slots are
+ * written before they are read and need no zeroing).  With only the minimum
+ * workspace the linears never split.  Depends on the current device's SM
+ * count.  Returns 0 for invalid arguments.
  */
 size_t convrot_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
 

@@ -318,6 +318,7 @@ struct GemmPlan {
     int bn = 256;       // MMA N: output features (token-major) or tokens (feature-major)
     int splits = 1;
     int64_t tiles = 0;
+    int streamk = 0;    // token-major stream-K: CTAs sharing the K steps of all tiles (0: off)
 };
 
 constexpr int kMaxSplitTiles = 512;              // split-K counters in a linear's workspace
@@ -325,6 +326,13 @@ constexpr size_t kCounterBytes = kMaxSplitTiles * 4;
 constexpr int64_t kSwapMaxTokens = 128;          // feature-major up to this many tokens
 constexpr int kSwapTokens = 32;                  // token tile of the feature-major GEMM
 constexpr int64_t kMaxSplitFeatures = 32768;     // split K only for N up to this
+// Stream-K: the cost of the shared tiles (148 partial tiles of 128 KB stored and
+// read back, ~5 us on B200), in 128-deep steps of a 256-wide tile: int8 weights
+// / widened int4 weights (whose steps are slower).  Measured, CUDA-graph-timed,
+// against the whole-tile plan: ViT-L widths at K = 1024 +5 us (int8 and int4),
+// K = 4096 N = 1024 +1.1 us (int8) and -4.2 us (int4).
+constexpr double kStreamKOverheadSteps8 = 16.0;
+constexpr double kStreamKOverheadSteps4 = 9.0;
 
 // Few tokens: feature-major tiles (128 features x 32 tokens), K split so that
 // the tiles x splits units cover the SMs (at most 8 slices, each at least 8
@@ -376,11 +384,30 @@ GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split, b
     // weights; with widened int4 weights pairs measured slower)
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
     p.pair = p.bn == 256 && !w4 && K >= 1536 && pair_tiles >= sms;
+    // Stream-K (needs the workspace's partial-tile slots): every SM takes an
+    // equal share of the K steps of all 256-wide tiles, so a partly filled last
+    // round of tiles costs nothing; each boundary between two SMs' shares
+    // costs one partial tile stored and read back.  Used where it beats the
+    // rounds of whole tiles (in 128-deep steps of a 256-wide tile) by 5 %,
+    // which takes deep K (int4 weights from K = 4096, int8 from ~8192).
+    const int64_t t256 = tiles_m * ((N + 255) / 256), nkb = K / 128;
+    if (allow_split && !p.pair && N >= 256 && sms < convrot::kStreamKFlags && t256 >= sms && t256 % sms != 0 &&
+        t256 * nkb < (int64_t(1) << 31)) {
+        const double sk = static_cast<double>(t256) * static_cast<double>(nkb) / sms +
+                          (w4 ? kStreamKOverheadSteps4 : kStreamKOverheadSteps8);
+        if (sk < 0.95 * best * static_cast<double>(nkb)) {
+            p.bn = 256;
+            p.tiles = t256;
+            p.streamk = sms;
+        }
+    }
     return p;
 }
 
-// int32 M x N sum buffer of a split feature-major GEMM.
+// int32 M x N sum buffer of a split feature-major GEMM, or the partial-tile
+// slots of a stream-K one (one 128 x BN int32 tile per boundary between CTAs).
 size_t split_buffer_bytes(const GemmPlan &p, int64_t M, int64_t N) {
+    if (p.streamk > 0) return static_cast<size_t>(p.streamk + 1) * 128 * p.bn * 4;
     return p.splits > 1 ? round256(static_cast<size_t>(M) * N * 4) : 0;
 }
 
@@ -390,7 +417,7 @@ template <class Cfg>
 convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, const void *Wc, int64_t M, int64_t N,
                                  int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
                                  int32_t *acc_out, cudaStream_t st, int splits, int32_t *acc_buf,
-                                 unsigned int *counters) {
+                                 unsigned int *counters, int streamk = 0) {
     {
         static std::mutex mu;
         static bool done[kMaxDevices] = {};
@@ -446,13 +473,15 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, cons
         launch_pdl_cluster(convrot::gemm_i8_tcgen05_kernel<Cfg>, dim3(static_cast<unsigned>(2 * clusters)),
                            dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, 2u, ta, tb, ty, static_cast<int>(rows_a),
                            static_cast<int>(rows_b), static_cast<int>(K), sx, sw, static_cast<const __half *>(bias),
-                           static_cast<__half *>(Y), acc_out, splits, acc_buf, counters);
+                           static_cast<__half *>(Y), acc_out, splits, acc_buf, counters, 0);
         return launch_status("gemm_i8_tcgen05 (CTA pairs)");
     }
-    const int grid = static_cast<int>(units < info->sms ? units : info->sms);
+    // persistent: one CTA per SM (stream-K: exactly the planned number of shares)
+    const int grid = streamk > 0 ? streamk : static_cast<int>(units < info->sms ? units : info->sms);
     launch_pdl(convrot::gemm_i8_tcgen05_kernel<Cfg>, dim3(grid), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, ta, tb,
                ty, static_cast<int>(rows_a), static_cast<int>(rows_b), static_cast<int>(K), sx, sw,
-               static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out, splits, acc_buf, counters);
+               static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out, splits, acc_buf, counters,
+               streamk);
     return launch_status("gemm_i8_tcgen05");
 }
 
@@ -494,6 +523,9 @@ convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const vo
     if (p.swap)
         return launch_gemm_cfg<GemmCfg<kSwapTokens, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y,
                                                                    acc_out, st, p.splits, acc_buf, counters);
+    if (p.streamk > 0)  // token-major, single CTAs, 256-wide tiles
+        return launch_gemm_cfg<GemmCfg<256, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
+                                                     acc_buf, counters, p.streamk);
     if (p.bn == 192)
         return launch_gemm_cfg<GemmCfg<192, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
                                                      nullptr, nullptr);
@@ -717,8 +749,9 @@ static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int
     if (workspace_bytes > base) {
         size_t cap;
         if (n_features >= 0) {
+            // (stream-K partial slots are written before they are read: only the counters)
             const GemmPlan p = plan_gemm(info->sms, M, n_features, K, true, bits == 4);
-            cap = kCounterBytes + split_buffer_bytes(p, M, n_features);
+            cap = kCounterBytes + (p.streamk > 0 ? 0 : split_buffer_bytes(p, M, n_features));
         } else {
             cap = kCounterBytes + (M <= kSwapMaxTokens ? round256(static_cast<size_t>(M) * kMaxSplitFeatures * 4) : 0);
         }
@@ -746,7 +779,8 @@ static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace
     // (which the activation half zeroed)
     GemmPlan p = plan_gemm(info->sms, M, N, K, true, bits == 4);
     const size_t base = convrot_workspace_bytes(M, K, bits) + kCounterBytes;
-    if (p.splits > 1 && workspace_bytes < base + split_buffer_bytes(p, M, N)) p.splits = 1;
+    if ((p.splits > 1 || p.streamk > 0) && workspace_bytes < base + split_buffer_bytes(p, M, N))
+        p = plan_gemm(info->sms, M, N, K, false, bits == 4);
     if (bits == 8)
         return launch_gemm<false, false>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st, p, acc_buf,
                                          counters);

@@ -77,6 +77,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     return true;
 }
 
+// Waits until the 32-bit word at `flag` (global memory, raised by another CTA
+// of the same grid with flag_raise) is nonzero; acquire ordering, bounded like
+// mbar_wait.
+__device__ __forceinline__ bool flag_wait(const unsigned int *flag, volatile int *abort) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v != 0u) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_device_status, kStatusTimeout);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+// Sets `flag` to 1 with release ordering (everything this thread has ordered
+// before becomes visible to a flag_wait that sees it).
+__device__ __forceinline__ void flag_raise(unsigned int *flag) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(1u) : "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {

@@ -39,6 +39,10 @@
 
 namespace convrot {
 
+// Stream-K ready flags live in the counters array from this index on (the
+// arrival counts below it): at most kStreamKFlags CTAs per stream-K grid.
+constexpr int kStreamKFlags = 256;
+
 // A4 / B4: the MMA's A / B operand arrives as packed int4 (two codes per byte)
 // and is widened in shared memory; otherwise it is int8 loaded by TMA straight
 // into the MMA ring.  Widened bytes hold 16 * code, so the accumulator carries
@@ -171,13 +175,17 @@ __device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[CHUN
 // rows of B).  Token-major: M = tokens, N = output features.  Feature-major:
 // M = output features, N = tokens.  sx is always the per-token scale, sw the
 // per-feature scale, bias per feature; Y and acc_out are tokens x features.
+// acc_buf / counters: the feature-major split-K sum buffer (M x N int32) and
+// per-tile counters; with streamk (token-major, single CTAs) the partial-tile
+// slots (TILE_M x BN int32 per CTA boundary) and per-boundary arrival counts
+// (counters[b]) and ready flags (counters[kStreamKFlags + b]).
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmY, int M, int N, int K, const float *__restrict__ sx,
                            const float *__restrict__ sw, const __half *__restrict__ bias, __half *__restrict__ Y,
                            int32_t *__restrict__ acc_out, int splits, int32_t *__restrict__ acc_buf,
-                           unsigned int *__restrict__ counters) {
+                           unsigned int *__restrict__ counters, int streamk) {
     constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, PSTAGES = Cfg::PSTAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -216,6 +224,37 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     auto unit_tile = [&](int u) { return u / splits; };
     auto unit_kb0 = [&](int u) { return (u - (u / splits) * splits) * num_kb / splits; };
     auto unit_kb1 = [&](int u) { return (u - (u / splits) * splits + 1) * num_kb / splits; };
+    // Stream-K (token-major, single CTAs): the tile-major sequence of (tile, K
+    // step) pairs, num_tiles * num_kb long, is cut into gridDim.x equal ranges
+    // (each at least num_kb long, so a tile is shared by at most two CTAs).  A
+    // range falls into segments: the last steps of a tile, whole tiles, the
+    // first steps of a tile.  Otherwise a segment is one work unit.
+    // (The host keeps num_tiles * num_kb below 2^31.)
+    const bool sk = !Cfg::SWAP && !Cfg::PAIR && streamk != 0;
+    const int64_t sk_total = static_cast<int64_t>(num_tiles) * num_kb;
+    const int sk_lo = sk ? static_cast<int>(sk_total * blockIdx.x / gridDim.x) : 0;
+    const int sk_hi = sk ? static_cast<int>(sk_total * (blockIdx.x + 1) / gridDim.x) : 0;
+    struct Seg {
+        int u;               // unit, or the range position of the segment's first step
+        int tile, kb0, kb1;  // tile < 0: no more work
+    };
+    auto seg_at = [&](int u) {
+        Seg g{u, -1, 0, 0};
+        if (sk) {
+            if (u < sk_hi) {
+                g.tile = u / num_kb;
+                g.kb0 = u - g.tile * num_kb;
+                g.kb1 = sk_hi - u < num_kb - g.kb0 ? g.kb0 + (sk_hi - u) : num_kb;
+            }
+        } else if (u < num_units) {
+            g.tile = unit_tile(u);
+            g.kb0 = unit_kb0(u);
+            g.kb1 = unit_kb1(u);
+        }
+        return g;
+    };
+    auto seg_first = [&]() { return seg_at(sk ? sk_lo : first_unit); };
+    auto seg_next = [&](const Seg &g) { return seg_at(sk ? g.u + (g.kb1 - g.kb0) : g.u + unit_stride); };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -273,10 +312,10 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             for (int i = 0; i < STAGES; ++i) filled[i] = false;
             for (int i = 0; i < PSTAGES; ++i) pfilled[i] = false;
             bool ok = true;
-            for (int unit = first_unit; ok && unit < num_units; unit += unit_stride) {
-                const int tile = unit_tile(unit);
+            for (Seg g = seg_first(); ok && g.tile >= 0; g = seg_next(g)) {
+                const int tile = g.tile;
                 const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
-                for (int kb = unit_kb0(unit); kb < unit_kb1(unit); ++kb) {
+                for (int kb = g.kb0; kb < g.kb1; ++kb) {
                     if (Cfg::TMA_RING) {
                         if (!mbar_wait(&empty[s], ph ^ 1, abort)) {
                             ok = false;
@@ -344,14 +383,14 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             uint32_t ph = 0;
             bool ok = true;
             int local = 0;
-            for (int unit = first_unit; ok && unit < num_units; unit += unit_stride, ++local) {
+            for (Seg g = seg_first(); ok && g.tile >= 0; g = seg_next(g), ++local) {
                 const int acc = local & 1;
                 const uint32_t acc_ph = (local >> 1) & 1;
                 if (!mbar_wait(&tmem_empty[acc], acc_ph ^ 1, abort)) break;
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * BN;
-                const int kb0 = unit_kb0(unit);
-                for (int kb = kb0; kb < unit_kb1(unit); ++kb) {
+                const int kb0 = g.kb0;
+                for (int kb = kb0; kb < g.kb1; ++kb) {
                     if (!mbar_wait(&full[s], ph, abort)) {
                         ok = false;
                         break;
@@ -409,16 +448,20 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         };
         float next_w;
         __half next_b;
-        load_scales(unit_tile(first_unit < num_units ? first_unit : 0), next_w, next_b);
+        {
+            const Seg g0 = seg_first();
+            load_scales(g0.tile >= 0 ? g0.tile : num_tiles, next_w, next_b);
+        }
         int local = 0;
-        int n_split_units = 0;  // split units handled so far (parity of the split-K barriers)
-        for (int unit = first_unit; unit < num_units; unit += unit_stride, ++local) {
-            const int tile = unit_tile(unit);
+        int n_split_units = 0;  // split units / shared tiles handled so far (parity of `decided`)
+        int n_partials = 0;     // stream-K partial tiles stored so far (parity of `partial_done`)
+        for (Seg g = seg_first(); g.tile >= 0; g = seg_next(g), ++local) {
+            const int tile = g.tile;
             const int acc = local & 1;
             const uint32_t acc_ph = (local >> 1) & 1;
             if (!mbar_wait_warp(&tmem_full[acc], acc_ph, abort)) break;
             tc_fence_after_sync();
-            // every epilogue thread is done with the previous unit's scales
+            // every epilogue thread is done with the previous segment's scales
             if (local > 0 && !mbar_wait_warp(scale_free, (local - 1) & 1, abort)) break;
             if (scol < BN) {
                 col_s[scol] = next_w;
@@ -426,7 +469,10 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             }
             mbar_arrive(scale_ready);
             if (!mbar_wait_warp(scale_ready, local & 1, abort)) break;
-            load_scales(unit + unit_stride < num_units ? unit_tile(unit + unit_stride) : num_tiles, next_w, next_b);
+            {
+                const Seg gn = seg_next(g);
+                load_scales(gn.tile >= 0 ? gn.tile : num_tiles, next_w, next_b);
+            }
             const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
             const int row0 = tm * Cfg::TILE_M + static_cast<int>(rank) * BM + q * 32;
             const int row = row0 + lane;
@@ -436,6 +482,37 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             constexpr int NCHUNK = Cfg::EPI_COLS / CH;
             if constexpr (!Cfg::SWAP) {
                 // ---- token-major: row = token; 32 x 32 boxes through shared memory and TMA
+                // Stream-K, a tile shared with the neighbouring CTA (boundary
+                // `slot`): the first of the two to get here stores its int32
+                // partial (fragment-major: warp, chunk, register, lane) in the
+                // boundary's slot and raises the slot's flag; the second waits
+                // for the flag (the first is running and only storing), adds the
+                // partial to its own and writes Y.  Integer addition is exact, so
+                // the result does not depend on which CTA comes first.
+                int sk_role = 0;  // 0: whole tile; 1: store the partial; 2: add the partial
+                int slot = 0;
+                int32_t *sk_part = nullptr;
+                if (sk && (g.kb0 != 0 || g.kb1 != num_kb)) {
+                    slot = g.kb0 != 0 ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) + 1;
+                    if (ew == 0 && lane == 0) {
+                        int role = 0;
+                        const unsigned int before = atomicAdd(&counters[slot], 1u);
+                        if (before == 0u) {
+                            role = 1;
+                        } else if (flag_wait(&counters[kStreamKFlags + slot], abort)) {
+                            counters[slot] = 0u;  // both arrived: ready for the next call
+                            counters[kStreamKFlags + slot] = 0u;
+                            role = 2;
+                        }
+                        *s_last = role;
+                        mbar_arrive(decided);
+                    }
+                    if (!mbar_wait_warp(decided, n_split_units & 1, abort)) break;
+                    ++n_split_units;
+                    sk_role = *s_last;
+                    if (sk_role == 0) break;  // abandoned after a timeout
+                    sk_part = acc_buf + static_cast<int64_t>(slot) * (Cfg::TILE_M * BN) + ew * (NCHUNK * 1024);
+                }
                 uint8_t *box = outbuf + ew * Cfg::OUT_BOX_BYTES;
                 const float sxm = row_ok ? sx[row] : 0.0f;
                 // 64-byte rows, 16-byte chunk g stored at g ^ ((row / 2) & 3) (64B swizzle)
@@ -449,13 +526,24 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     tmem_ld_32x32(tbase + col_local, r);
                     tmem_ld_wait();
                     if (c == NCHUNK - 1) {
-                        // every TMEM read of this unit by this thread is complete
+                        // every TMEM read of this segment by this thread is complete
                         tc_fence_before_sync();
                         if (Cfg::PAIR) mbar_arrive_cluster(cluster_addr(&tmem_empty[acc], 0));
                         else mbar_arrive(&tmem_empty[acc]);
                     }
                     const int col0 = tn * BN + col_local;
                     if (row0 >= M || col0 >= N) continue;  // whole box outside Y (warp-uniform)
+                    if (sk_role == 1) {
+                        int32_t *dst = sk_part + c * 1024 + lane;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) __stcg(dst + 32 * j, static_cast<int32_t>(r[j]));
+                        continue;
+                    }
+                    if (sk_role == 2) {
+                        const int32_t *src = sk_part + c * 1024 + lane;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) r[j] += static_cast<uint32_t>(__ldcg(src + 32 * j));
+                    }
                     // the store issued from this box last time must have read it
                     if (lane == 0) bulk_wait_group_read<0>();
                     __syncwarp();
@@ -492,6 +580,16 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                         tma_store_2d(&tmY, box, col0, row0);
                         bulk_commit_group();
                     }
+                }
+                if (sk_role == 1) {
+                    // every thread's partial is visible device-wide before the flag goes up
+                    __threadfence();
+                    mbar_arrive(partial_done);
+                    if (ew == 0 && lane == 0 && mbar_wait(partial_done, n_partials & 1, abort)) {
+                        __threadfence();
+                        flag_raise(&counters[kStreamKFlags + slot]);
+                    }
+                    ++n_partials;
                 }
             } else {
                 // ---- feature-major: row = output feature f, columns = tokens
@@ -573,8 +671,8 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         int ps = 0, us = 0;
         uint32_t pph = 0, uph = 0;
         bool ok = true;
-        for (int unit = first_unit; ok && unit < num_units; unit += unit_stride) {
-            for (int kb = unit_kb0(unit); kb < unit_kb1(unit); ++kb) {
+        for (Seg g = seg_first(); ok && g.tile >= 0; g = seg_next(g)) {
+            for (int kb = g.kb0; kb < g.kb1; ++kb) {
                 if (!mbar_wait_warp(&pfull[ps], pph, abort) || !mbar_wait_warp(&empty[us], uph ^ 1, abort)) {
                     ok = false;
                     break;

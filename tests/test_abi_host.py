@@ -122,8 +122,20 @@ def test_linear_workspace_bytes_adds_split_k_room(lib):
     # the weight-streaming kernel (one token) needs no split state beyond the counters
     assert lws(1, 4096, 4096, 8) == ws(1, 4096, 8) + 2048
     assert lws(8, 4096, 4096, 4) == ws(8, 4096, 4) + 2048
-    # thousands of output tiles: no split, only the counters
+    # thousands of output tiles on CTA pairs: no split, only the counters
     assert lws(16384, 4096, 4096, 8) == ws(16384, 4096, 8) + 2048
+    # token-major stream-K (deep K, a partly filled last round of 128 x 256 tiles):
+    # one 128 x 256 int32 partial-tile slot per boundary between the 148 shares (+1)
+    slots = 149 * 128 * 256 * 4
+    assert lws(5184, 4096, 1024, 4) == ws(5184, 4096, 4) + 2048 + slots
+    for bits in (8, 4):
+        assert lws(2500, 8192, 2000, bits) == ws(2500, 8192, bits) + 2048 + slots
+    # shallow K (the shared tiles cost more than the idle SMs): whole tiles, counters only
+    for K, N in [(1024, 3072), (1024, 1024), (1024, 4096)]:
+        assert lws(5184, K, N, 8) == ws(5184, K, 8) + 2048
+    assert lws(5184, 4096, 1024, 8) == ws(5184, 4096, 8) + 2048
+    # a whole number of rounds of tiles (148 x 2 = 296 = 37 x 8 tiles): no stream-K
+    assert lws(37 * 128, 8192, 8 * 256, 8) == ws(37 * 128, 8192, 8) + 2048
     assert lws(-1, 4096, 4096, 8) == 0
     assert lws(4, 4096, 4096, 5) == 0
 

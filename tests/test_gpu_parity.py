@@ -323,15 +323,21 @@ def test_linear_two_stage_entry_points_equal_the_linear(bits):
     assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
 
 
-SPLIT_CASES = [(1, 4096, 4096), (16, 4096, 4096), (100, 1024, 4096), (700, 1024, 4096), (5184, 1024, 4096)]
+# (M, N, K): the feature-major split (M <= 128); the token-major stream-K plan
+# (5184 x 1024 x 4096 with int4 weights; 2500 x 2000 x 8192, ragged M and N,
+# with both widths); the whole-tile plan with the larger workspace
+SPLIT_CASES = [(1, 4096, 4096), (16, 4096, 4096), (100, 1024, 4096), (700, 1024, 4096), (5184, 1024, 4096),
+               (2500, 2000, 8192), (5184, 3072, 1024)]
 
 
 @pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("M,N,K", SPLIT_CASES)
 def test_linear_split_k_bit_exact(M, N, K, bits):
-    """With the larger workspace the linear may split K across CTAs; the int32
-    sum of the slices is exact, so the output equals the unsplit linear's and
-    the oracle's GEMM of the same codes, bit for bit, on every call."""
+    """With the larger workspace the linear may split K across CTAs (feature-major
+    K slices, or token-major stream-K shares whose boundary tiles are summed
+    from two CTAs' partials); the int32 sums are exact, so the output equals the
+    unsplit linear's and the oracle's GEMM of the same codes, bit for bit, on
+    every call (the split state resets itself between calls)."""
     X = wl.activations(M, K, 0.01, 30.0, seed=M + 7)
     W = wl.weight(N, K, 0.02, seed=N + 7)
     bias = wl.bias(N, seed=3)
