@@ -523,9 +523,11 @@ convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const vo
     if (p.swap)
         return launch_gemm_cfg<GemmCfg<kSwapTokens, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y,
                                                                    acc_out, st, p.splits, acc_buf, counters);
-    if (p.streamk > 0)  // token-major, single CTAs, 256-wide tiles
-        return launch_gemm_cfg<GemmCfg<256, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
-                                                     acc_buf, counters, p.streamk);
+    if constexpr (!X4) {  // (stream-K needs a linear's workspace, whose activation codes are bytes)
+        if (p.streamk > 0)  // token-major, single CTAs, 256-wide tiles
+            return launch_gemm_cfg<GemmCfg<256, false, W4, false, false, true>>(
+                info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1, acc_buf, counters, p.streamk);
+    }
     if (p.bn == 192)
         return launch_gemm_cfg<GemmCfg<192, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
                                                      nullptr, nullptr);

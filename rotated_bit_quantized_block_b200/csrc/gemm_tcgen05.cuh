@@ -49,7 +49,8 @@ constexpr int kStreamKFlags = 256;
 // a factor 16 per widened operand (ACC_SHIFT undoes it).
 // PAIR: a cluster of two CTAs shares each 256 x BN tile through one
 // cta_group::2 MMA (each CTA loads and keeps 128 rows of A and BN/2 rows of B).
-template <int BN_, bool A4_, bool B4_, bool SWAP_ = false, bool PAIR_ = false>
+// SK: token-major stream-K (equal shares of all tiles' K steps per CTA).
+template <int BN_, bool A4_, bool B4_, bool SWAP_ = false, bool PAIR_ = false, bool SK_ = false>
 struct GemmCfg {
     static constexpr int BM = 128;   // rows of A per CTA
     static constexpr int BN = BN_;   // accumulator columns
@@ -58,6 +59,7 @@ struct GemmCfg {
     static constexpr bool B4 = B4_;
     static constexpr bool SWAP = SWAP_;
     static constexpr bool PAIR = PAIR_;
+    static constexpr bool SK = SK_;
     static constexpr int CTAS = PAIR ? 2 : 1;      // CTAs per tile
     static constexpr int TILE_M = BM * CTAS;       // accumulator rows per tile
     static constexpr int B_ROWS = BN / CTAS;       // rows of B held by one CTA
@@ -104,6 +106,7 @@ struct GemmCfg {
     static constexpr uint32_t IDESC = idesc_i8(TILE_M, BN);
     static_assert(STAGES >= 2, "pipeline depth");
     static_assert(!PAIR || (!SWAP && !A4 && !B4 && BN == 256), "CTA pairs: token-major W8A8, 256-wide tiles");
+    static_assert(!SK || (!SWAP && !PAIR), "stream-K: token-major, single CTAs");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
     static_assert(SWAP ? (BN == 32 || BN == 64 || BN == 128 || BN == 256) : (BN % 64 == 0 && BN >= 64 && BN <= 256),
                   "tile width");
@@ -176,9 +179,9 @@ __device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[CHUN
 // M = output features, N = tokens.  sx is always the per-token scale, sw the
 // per-feature scale, bias per feature; Y and acc_out are tokens x features.
 // acc_buf / counters: the feature-major split-K sum buffer (M x N int32) and
-// per-tile counters; with streamk (token-major, single CTAs) the partial-tile
-// slots (TILE_M x BN int32 per CTA boundary) and per-boundary arrival counts
-// (counters[b]) and ready flags (counters[kStreamKFlags + b]).
+// per-tile counters; with streamk (Cfg::SK) the partial-tile slots (TILE_M x BN
+// int32 per CTA boundary) and per-boundary arrival counts (counters[b]) and
+// ready flags (counters[kStreamKFlags + b]).
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     // range falls into segments: the last steps of a tile, whole tiles, the
     // first steps of a tile.  Otherwise a segment is one work unit.
     // (The host keeps num_tiles * num_kb below 2^31.)
-    const bool sk = !Cfg::SWAP && !Cfg::PAIR && streamk != 0;
+    const bool sk = Cfg::SK && streamk != 0;
     const int64_t sk_total = static_cast<int64_t>(num_tiles) * num_kb;
     const int sk_lo = sk ? static_cast<int>(sk_total * blockIdx.x / gridDim.x) : 0;
     const int sk_hi = sk ? static_cast<int>(sk_total * (blockIdx.x + 1) / gridDim.x) : 0;
