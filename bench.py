@@ -2,9 +2,12 @@
 
 One step = one pass of the whole online path (rotate + per-token quantize +
 integer GEMM + dequant) over every linear of the workload, for one batch of M
-synthetic tokens.  Default workload: the W8A8 ViT-L encoder linears (qkv
-1024->3072, proj 1024->1024, fc1 1024->4096, fc2 4096->1024) at M = 5184 tokens
-(72 x 72 patches), Hadamard block 128.
+synthetic tokens, through the public linear entry points (one fused launch per
+linear where the plan allows).  Default workload: the W8A8 DiT linears (qkv
+1536->4608, fc1 1536->6144, fc2 6144->1536) at M = 8192 tokens (batch 2 x 4096),
+Hadamard block 128 -- the largest configuration.  The same JSON line carries
+sub-results for the ViT-L W8A8 / W4A4 / mixed-width linears and the M sweep,
+and context rows (cuBLAS fp16 linear, torch._int_mm ceiling).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
@@ -165,10 +168,20 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------------------ workload
 
-class Replica:
-    """Device buffers of one independent batch: per linear X, Y, codes, workspace."""
+def set_count(w: wl.Workload) -> int:
+    """Rotating buffer sets so that one pass over all of them moves more than
+    1.5 x L2 (weights, X, Y and workspaces): no timed step finds its inputs in L2."""
+    per_set = 0
+    for lin in w.linears:
+        b = w.bits_of(lin)
+        per_set += lin.N * lin.K * b // 8 + 2 * w.M * lin.K + 2 * w.M * lin.N + w.M * lin.K
+    return max(2, min(16, -(-int(1.5 * L2_BYTES) // max(per_set, 1))))
 
-    def __init__(self, w: wl.Workload, replica: int, device):
+
+class Replica:
+    """Device buffers of one independent batch: per linear X, Y, weights and workspace."""
+
+    def __init__(self, w: wl.Workload, replica: int, device, host_copies: bool = False):
         self.items = []
         for i, lin in enumerate(w.linears):
             X, W, _ = wl.linear_inputs(w, i, replica=replica)
@@ -176,38 +189,52 @@ class Replica:
             Wd = torch.from_numpy(W).to(device)
             Wq, sw = cr.convrot_quantize_weight(Wd, w.block, w.bits_of(lin), cr.CLIP_MSE)
             need = cr.convrot_linear_workspace_bytes(w.M, lin.K, lin.N, w.bits_of(lin))
-            self.items.append({
-                "lin": lin, "X": Xd, "Xhost": torch.from_numpy(X).pin_memory(), "Wq": Wq, "sw": sw,
-                "Y": torch.empty((w.M, lin.N), dtype=torch.float16, device=device),
-                "Yhost": torch.empty((w.M, lin.N), dtype=torch.float16).pin_memory(),
-                "ws": torch.empty(need, dtype=torch.uint8, device=device),
-                "W": Wd,
-            })
+            item = {"lin": lin, "X": Xd, "Wq": Wq, "sw": sw, "W": Wd,
+                    "Y": torch.empty((w.M, lin.N), dtype=torch.float16, device=device),
+                    "ws": torch.empty(need, dtype=torch.uint8, device=device)}
+            if host_copies:
+                item["Xhost"] = torch.from_numpy(X).pin_memory()
+                item["Yhost"] = torch.empty((w.M, lin.N), dtype=torch.float16).pin_memory()
+            self.items.append(item)
 
     def nbytes(self):
         return sum(it["X"].nbytes + it["Y"].nbytes + it["Wq"].nbytes + it["ws"].nbytes for it in self.items)
 
 
-def run_step(w, rep, stream, events=None):
-    """One pass over every linear: rotate+quant kernel, then GEMM+dequant kernel.
+def linear_call(w, it, stream):
+    """One linear through the public entry point (one fused launch where the plan allows)."""
+    fn = cr.convrot_linear_w8a8 if w.bits_of(it["lin"]) == 8 else cr.convrot_linear_w4a4
+    fn(it["X"], it["Wq"], it["sw"], w.block, None, it["Y"], it["ws"], stream)
 
-    The two kernels are launched through convrot_linear_quant_act and
-    convrot_linear_gemm, the two halves of convrot_linear_*.  With ``events`` (per linear: act start,
-    act end = GEMM start, GEMM end) every kernel is bracketed for per-kernel
-    timing; event nodes between kernels also stop the next kernel from starting
-    early, so the throughput pass runs without them.
-    """
-    for i, it in enumerate(rep.items):
-        lin = it["lin"]
-        ws = it["ws"]
-        if events is not None:
-            events[i][0].record(stream)
-        cr.convrot_linear_quant_act(it["X"], w.block, w.bits_of(lin), ws, stream=stream)
-        if events is not None:
-            events[i][1].record(stream)
-        cr.convrot_linear_gemm(ws, w.M, lin.K, w.bits_of(lin), it["Wq"], it["sw"], None, it["Y"], stream=stream)
-        if events is not None:
-            events[i][2].record(stream)
+
+def run_step(w, rep, stream):
+    """One pass over every linear of the workload for one batch of tokens."""
+    for it in rep.items:
+        linear_call(w, it, stream)
+
+
+def graph_ms(calls, stream, reps: int = 3) -> float:
+    """Average device time of one call of ``calls`` (a list of callables taking a
+    stream), captured back to back in one CUDA graph and replayed: events on the
+    launching stream around the replay; best of ``reps`` replays."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for c in calls:
+            c(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()  # untimed
+        torch.cuda.synchronize()
+        best = None
+        for _ in range(reps):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / len(calls)
+            best = t if best is None else min(best, t)
+    del g
+    return best
 
 
 def run_e2e(w, reps, stream, steps):
@@ -224,7 +251,7 @@ def run_e2e(w, reps, stream, steps):
     s_in.wait_stream(stream)
     s_out.wait_stream(stream)
     for s in range(steps):
-        r = s % 2
+        r = s % len(reps)
         for i, it in enumerate(reps[r].items):
             key = (r, i)
             if key in consumed:
@@ -236,8 +263,7 @@ def run_e2e(w, reps, stream, steps):
             stream.wait_event(uploaded)
             if key in downloaded:
                 stream.wait_event(downloaded[key])
-            fn = cr.convrot_linear_w8a8 if w.bits_of(it["lin"]) == 8 else cr.convrot_linear_w4a4
-            fn(it["X"], it["Wq"], it["sw"], w.block, None, it["Y"], it["ws"], stream)
+            linear_call(w, it, stream)
             done = torch.cuda.Event()
             done.record(stream)
             consumed[key] = done
@@ -271,12 +297,13 @@ def oracle_weights(w: wl.Workload):
     return _ORACLE_WEIGHTS[w.name]
 
 
-def time_oracle(w: wl.Workload, budget_s: float, max_rows: int | None = None):
+def time_oracle(w: wl.Workload, budget_s: float, max_rows: int | None = None, threads: int | None = None):
     """Times the CPU oracle (rotate+quant, integer GEMM, dequant) on a bounded
-    sample of rows of every linear of the workload."""
+    sample of rows of every linear of the workload (all host cores unless
+    ``threads`` is given)."""
     import oracle  # the oracle is only used by the CPU baseline legs
 
-    threads = oracle.set_threads(os.cpu_count() or 1)
+    threads = oracle.set_threads(threads or os.cpu_count() or 1)
     weights = oracle_weights(w)
 
     def run(rows):
@@ -364,6 +391,172 @@ def config_of(w: wl.Workload):
     }
 
 
+def linear_bytes(w, lin, M=None) -> int:
+    """Algorithmic bytes of one linear with the rotate+quant fused in: X read,
+    codes in and out of L2 are not counted, weights, Y and scales."""
+    M = w.M if M is None else M
+    return 2 * M * lin.K + lin.N * lin.K * w.bits_of(lin) // 8 + 2 * M * lin.N + 4 * M + 4 * lin.N
+
+
+def act_bytes(w, lin) -> int:
+    """Algorithmic bytes of the activation pass: X read, one code byte per element and the scales written."""
+    return 3 * w.M * lin.K + 4 * w.M
+
+
+def measure_workload(w, reps, stream, steps, peaks, clock_index=None, warmup=3):
+    """Times one workload: ``warmup`` eager steps, then the step graph (``steps``
+    steps over rotating buffer sets, the value), then every linear by itself
+    (the public linear, and its two halves apart) in graphs of back-to-back
+    launches over the same sets."""
+    n_sets = len(reps)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for s in range(warmup):
+            run_step(w, reps[s % n_sets], stream)
+    torch.cuda.synchronize()
+    cr.convrot_device_status(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for s in range(steps):
+            run_step(w, reps[s % n_sets], stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = None
+    with torch.cuda.stream(stream):
+        g.replay()  # untimed
+        torch.cuda.synchronize()
+        if clock_index is not None:
+            with ClockSampler(clock_index) as clk:
+                start.record(stream)
+                g.replay()
+                end.record(stream)
+                torch.cuda.synchronize()
+            clocks = clk.summary()
+        else:
+            start.record(stream)
+            g.replay()
+            end.record(stream)
+            torch.cuda.synchronize()
+    del g
+    elapsed_ms = start.elapsed_time(end)
+    cr.convrot_device_status(stream)
+
+    per = {}
+    for i, lin in enumerate(w.linears):
+        bits = w.bits_of(lin)
+        items = [rep.items[i] for rep in reps]
+        plan = cr.convrot_linear_plan(w.M, lin.K, lin.N, bits, w.block, items[0]["ws"].numel())
+        calls = [(lambda st, it=it: linear_call(w, it, st)) for it in items] * 2
+        act = [(lambda st, it=it: cr.convrot_linear_quant_act(it["X"], w.block, bits, it["ws"], stream=st))
+               for it in items] * 2
+        gemm = [(lambda st, it=it: cr.convrot_linear_gemm(it["ws"], w.M, lin.K, bits, it["Wq"], it["sw"], None,
+                                                          it["Y"], stream=st)) for it in items] * 2
+        t_lin, t_act, t_gemm = graph_ms(calls, stream), graph_ms(act, stream), graph_ms(gemm, stream)
+        per[lin.name] = {"plan": plan, "linear_ms": t_lin, "act_ms": t_act, "gemm_ms": t_gemm}
+    cr.convrot_device_status(stream)
+
+    ops = w.ops()
+    lin_ms = sum(v["linear_ms"] for v in per.values())
+    # the dominant kernel: the fused linear kernel where a linear is one launch,
+    # otherwise its GEMM (the activation launch is reported under rotate_quant)
+    dom_ms = sum(v["linear_ms"] if v["plan"]["fused"] else v["gemm_ms"] for v in per.values())
+    int8_peak = 2.0 * peaks["bf16_tflops"]  # dense int8 = 2 x dense bf16 (4.5 vs 2.25 POPS nominal)
+    if all(v["plan"]["gemm_kind"] == 2 for v in per.values()):
+        # the fewest tokens: bound by reading the weights; the fused kernel also
+        # reads X, the unfused one the activation codes
+        moved = sum(linear_bytes(w, l) - (0 if per[l.name]["plan"]["fused"] else w.M * l.K) for l in w.linears)
+        achieved = moved / (dom_ms / 1e3) / 1e9
+        fused = all(v["plan"]["fused"] for v in per.values())
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"],
+                "kernel": ("gemv_fused (rotate+quant in every CTA, weight-streaming dp4a)" if fused
+                           else "gemv_i8 (weight-streaming, dp4a)"),
+                "peak_note": f"{peaks['source']} HBM copy bandwidth"}
+    else:
+        achieved = ops / (dom_ms / 1e3) / 1e12
+        fused = all(v["plan"]["fused"] for v in per.values())
+        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
+                "frac": achieved / int8_peak,
+                "kernel": ("gemm_i8_tcgen05 with the fused rotate+quant prologue (int8 x int8 -> int32 in TMEM, "
+                           "dequant epilogue)" if fused else "gemm_i8_tcgen05 (int8 x int8 -> int32, dequant epilogue)"),
+                "peak_note": f"dense int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s"}
+    roof.update({
+        "timing": "each linear alone: CUDA graph of back-to-back launches over the rotating buffer sets, "
+                  "CUDA events on the launching stream around the replay",
+        "per_linear_us": {n: round(1e3 * (v["linear_ms"] if v["plan"]["fused"] else v["gemm_ms"]), 2)
+                          for n, v in per.items()},
+        "per_linear_frac": {l.name: round(2 * w.M * l.K * l.N / ((per[l.name]["linear_ms"] if per[l.name]["plan"]["fused"]
+                                                                   else per[l.name]["gemm_ms"]) / 1e3) / 1e12
+                                          / int8_peak, 3) for l in w.linears},
+    })
+    act_total_ms = sum(v["act_ms"] for v in per.values())
+    act_gbs = sum(act_bytes(w, l) for l in w.linears) / (act_total_ms / 1e3) / 1e9
+    rq = {"bound": "hbm", "achieved": act_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+          "frac": act_gbs / peaks["hbm_gbs"],
+          "kernel": "act_rotate_quant_tma (the activation launch of the two-launch linear; fused into the GEMM "
+                    "otherwise)",
+          "algorithmic_bytes_per_linear": {l.name: act_bytes(w, l) for l in w.linears},
+          "per_linear_us": {n: round(1e3 * v["act_ms"], 2) for n, v in per.items()},
+          "per_linear_gbs": {l.name: round(act_bytes(w, l) / (per[l.name]["act_ms"] / 1e3) / 1e9, 1)
+                             for l in w.linears}}
+    return {
+        "elapsed_ms": elapsed_ms, "ms_per_step": elapsed_ms / steps, "clocks": clocks,
+        "tokens_per_s": w.M * steps / (elapsed_ms / 1e3), "tops": ops * steps / (elapsed_ms / 1e3) / 1e12,
+        "roofline": roof, "rotate_quant": rq,
+        "kernel_us_per_step": round(1e3 * lin_ms, 2),
+        "two_launch_us_per_step": round(1e3 * sum(v["act_ms"] + v["gemm_ms"] for v in per.values()), 2),
+        "launches_per_step": sum(v["plan"]["launches"] for v in per.values()),
+        "plans": {n: v["plan"] for n, v in per.items()},
+    }
+
+
+def eager_ms(fn, stream, reps: int = 20) -> float:
+    """Average device time of ``fn()`` launched ``reps`` times back to back on
+    ``stream`` (library calls that are not captured into graphs here)."""
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def context_rows(w, reps, stream, peaks):
+    """Context only: cuBLAS fp16 F.linear on the same shapes (over the same
+    rotating buffer sets), and a torch._int_mm 8192^3 int8 ceiling."""
+    out = {}
+    try:
+        per = {}
+        for i, lin in enumerate(w.linears):
+            pairs = [(rep.items[i]["X"], rep.items[i]["W16"]) for rep in reps]
+            k = [0]
+
+            def call(pairs=pairs, k=k):
+                X, W = pairs[k[0] % len(pairs)]
+                k[0] += 1
+                torch.nn.functional.linear(X, W)
+            per[lin.name] = round(1e3 * eager_ms(call, stream), 2)
+        out["f_linear_fp16_us"] = per
+        out["f_linear_fp16_us_per_step"] = round(sum(per.values()), 2)
+    except Exception as e:  # context only
+        out["f_linear_fp16_error"] = repr(e)[:200]
+    try:
+        n = 8192
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=stream.device)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=stream.device)
+        ms = eager_ms(lambda: torch._int_mm(a, b), stream, reps=10)
+        out["int_mm_8192_tops"] = round(2 * n ** 3 / (ms / 1e3) / 1e12, 1)
+        out["int_mm_8192_frac_of_int8_peak"] = round(2 * n ** 3 / (ms / 1e3) / 1e12 / (2 * peaks["bf16_tflops"]), 3)
+        del a, b
+    except Exception as e:
+        out["int_mm_error"] = repr(e)[:200]
+    return out
+
+
 def ours_arm(args, w, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -371,14 +564,14 @@ def ours_arm(args, w, rank, world, local_rank):
     peaks = load_peaks()
     stream = torch.cuda.Stream(device)
 
-    # offline conversion (timed once, reported separately; not part of a step)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    reps = [Replica(w, replica=r, device=device) for r in replica_ids(rank)]
+    n_sets = set_count(w)
+    reps = [Replica(w, replica=r, device=device, host_copies=True) for r in replica_ids(rank, n_sets)]
     torch.cuda.synchronize()
     setup_s = time.perf_counter() - t0
     per_set = reps[0].nbytes()
-    # offline weight conversion time, measured by itself
+    # offline weight conversion, measured by itself (not part of a step)
     wq_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     with torch.cuda.stream(stream):
         wq_ev[0].record(stream)
@@ -389,56 +582,15 @@ def ours_arm(args, w, rank, world, local_rank):
     weight_quant_ms = wq_ev[0].elapsed_time(wq_ev[1])
     for rep in reps:
         for it in rep.items:
-            del it["W"]
+            it["W16"] = it.pop("W")
 
-    # warm-up (eager), also initializes per-device kernel attributes before capture
-    with torch.cuda.stream(stream):
-        for s in range(args.warmup):
-            run_step(w, reps[s % 2], stream)
-    torch.cuda.synchronize()
-    cr.convrot_device_status(stream)
-
-    # capture the K timed steps twice: as they run (throughput), and with events
-    # around every kernel (per-kernel durations for the rooflines)
-    n_lin = len(w.linears)
-    events = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(n_lin)]
-              for _ in range(args.steps)]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for s in range(args.steps):
-            run_step(w, reps[s % 2], stream)
-    graph_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_ev, stream=stream):
-        for s in range(args.steps):
-            run_step(w, reps[s % 2], stream, events=events[s])
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        graph.replay()  # untimed replays of the captured steps
-        graph_ev.replay()
-    torch.cuda.synchronize()
-
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(device.index) as clk, torch.cuda.stream(stream):
-        start.record(stream)
-        graph.replay()
-        end.record(stream)
-        torch.cuda.synchronize()
-        graph_ev.replay()
-        torch.cuda.synchronize()
+    m = measure_workload(w, reps, stream, args.steps, peaks, clock_index=device.index, warmup=args.warmup)
     if world > 1:
         torch.distributed.barrier()
-    elapsed_ms = start.elapsed_time(end)
-    act_ms = [[events[s][i][0].elapsed_time(events[s][i][1]) for i in range(n_lin)] for s in range(args.steps)]
-    gemm_ms = [[events[s][i][1].elapsed_time(events[s][i][2]) for i in range(n_lin)] for s in range(args.steps)]
-    cr.convrot_device_status(stream)
-    clocks = clk.summary()
-
-    elapsed_ms = max_over_ranks(elapsed_ms, world, device)
-    ms_per_step = elapsed_ms / args.steps
-    tokens = w.M * world * args.steps
+    elapsed_ms = max_over_ranks(m["elapsed_ms"], world, device)
     value = whole_job_tokens_per_s(w.M, world, args.steps, elapsed_ms)
 
     # end to end through the public entry point, host buffers in pinned memory
@@ -448,8 +600,6 @@ def ours_arm(args, w, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    # the K steps (copies included) captured once, so that host-side launch
-    # cost does not stand in for the device's copy and compute time
     graph_e2e = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_e2e, stream=stream):
         run_e2e(w, reps, stream, args.steps)
@@ -460,6 +610,7 @@ def ours_arm(args, w, rank, world, local_rank):
         graph_e2e.replay()
         e_end.record(stream)
     torch.cuda.synchronize()
+    del graph_e2e
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, device)
     if world > 1:
         torch.distributed.barrier()
@@ -468,71 +619,60 @@ def ours_arm(args, w, rank, world, local_rank):
 
     if rank != 0:
         return
-    ops_step = w.ops()
-    gemm_total_ms = sum(sum(r) for r in gemm_ms)
-    gemm_ops_total = ops_step * args.steps
-    achieved_tops = gemm_ops_total / (gemm_total_ms / 1000.0) / 1e12
-    int8_peak = 2.0 * peaks["bf16_tflops"]  # dense int8 = 2 x dense bf16 (4.5 vs 2.25 POPS nominal)
-    per_linear_ms = [statistics.mean(gemm_ms[s][i] for s in range(args.steps)) for i in range(n_lin)]
-    per_linear_act_ms = [statistics.mean(act_ms[s][i] for s in range(args.steps)) for i in range(n_lin)]
     traffic = load_traffic(w.name)
-    gemm_traffic = traffic["gemm"]
-    gemm_bytes = {l.name: w.M * l.K + l.N * l.K * w.bits_of(l) // 8 + 2 * w.M * l.N + 4 * w.M + 4 * l.N
-                  for l in w.linears}
-    if all(weight_streaming(w.M, w.bits_of(l)) for l in w.linears):
-        # the fewest tokens run the weight-streaming GEMM: bound by reading the weights
-        achieved = sum(gemm_bytes.values()) * args.steps / (gemm_total_ms / 1000.0) / 1e9
-        bound = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                 "frac": achieved / peaks["hbm_gbs"], "kernel": "gemv_i8 (weight-streaming, dp4a)",
-                 "peak_note": f"{peaks['source']} HBM copy bandwidth"}
-    else:
-        bound = {"bound": "tensor", "achieved": achieved_tops, "peak": int8_peak, "unit": "TOPS",
-                 "frac": achieved_tops / int8_peak,
-                 "kernel": "gemm_i8_tcgen05 (int8 x int8 -> int32, fused dequant epilogue)",
-                 "peak_note": f"dense int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s"}
-    roofline = {
-        **bound,
-        # mean DRAM bytes per GEMM launch of one step, from the committed ncu capture
-        "traffic": (statistics.mean(gemm_traffic.values()) if gemm_traffic else None),
-        "traffic_per_linear": gemm_traffic,
-        "algorithmic_bytes_per_linear": gemm_bytes,
-        "timing": "second timed pass of the same steps with CUDA events around every kernel launch",
-        "per_linear_ms": {l.name: round(t, 5) for l, t in zip(w.linears, per_linear_ms)},
-        "per_linear_tops": {l.name: round(2 * w.M * l.K * l.N / (t / 1000) / 1e12, 1)
-                            for l, t in zip(w.linears, per_linear_ms)},
-    }
-    act_bytes = [w.M * l.K * 2 + w.M * l.K + 4 * w.M for l in w.linears]  # codes one byte each in the linear
-    act_total_ms = sum(per_linear_act_ms)
-    act_gbs = sum(act_bytes) / (act_total_ms / 1000.0) / 1e9
-    act_traffic = traffic["act"]
-    rotate_quant = {
-        "bound": "hbm", "achieved": act_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-        "frac": act_gbs / peaks["hbm_gbs"], "kernel": "act_rotate_quant",
-        "traffic": (statistics.mean(act_traffic.values()) if act_traffic else None),
-        "traffic_per_linear": act_traffic,
-        "algorithmic_bytes_per_linear": {l.name: b for l, b in zip(w.linears, act_bytes)},
-        "per_linear_ms": {l.name: round(t, 5) for l, t in zip(w.linears, per_linear_act_ms)},
-        "per_linear_gbs": {l.name: round(b / (t / 1000) / 1e9, 1)
-                           for l, b, t in zip(w.linears, act_bytes, per_linear_act_ms)},
-    }
+    roofline = dict(m["roofline"])
+    roofline["traffic"] = statistics.mean(traffic["gemm"].values()) if traffic["gemm"] else None
+    roofline["traffic_per_linear"] = traffic["gemm"]
+    roofline["algorithmic_bytes_per_linear"] = {l.name: linear_bytes(w, l) for l in w.linears}
+    rotate_quant = dict(m["rotate_quant"])
+    rotate_quant["traffic"] = statistics.mean(traffic["act"].values()) if traffic["act"] else None
+    rotate_quant["traffic_per_linear"] = traffic["act"]
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": dtype_of(w), "data": "synthetic",
-        "config": dict(config_of(w), l2=f"inputs larger than L2: 2 rotating buffer sets of "
+        "config": dict(config_of(w), l2=f"inputs larger than L2: {n_sets} rotating buffer sets of "
                                         f"{per_set / 2**20:.0f} MiB each (L2 {L2_BYTES >> 20} MiB)"),
-        "tops": ops_step * world * args.steps / (elapsed_ms / 1000.0) / 1e12,
+        "tops": m["tops"] * world,
         "roofline": roofline,
         "rotate_quant": rotate_quant,
+        "kernel_us_per_step": m["kernel_us_per_step"],
+        "two_launch_us_per_step": m["two_launch_us_per_step"],
+        "plans": m["plans"],
         "offline_weight_quant_ms": weight_quant_ms,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "convrot_linear_* with pinned-host X copied in and Y copied out every step "
                         "(uploads and downloads on their own streams, overlapping the linears; the K steps "
                         "replayed from one CUDA graph)"},
-        "gpu_launches": 2 * n_lin * args.steps,
-        "clocks": clocks,
+        "gpu_launches": m["launches_per_step"] * args.steps,
+        "clocks": m["clocks"],
         "setup_s": setup_s,
     }
+    if world == 1 and not args.no_sub_results:
+        subs = {}
+        for name in SUB_WORKLOADS:
+            if name == w.name:
+                continue
+            sw_ = workload_by_name(name)
+            sreps = [Replica(sw_, replica=r, device=device) for r in range(set_count(sw_))]
+            sm = measure_workload(sw_, sreps, stream, args.sub_steps, peaks)
+            subs[name] = {
+                "tokens_per_s": sm["tokens_per_s"], "tops": sm["tops"], "us_per_step": 1e3 * sm["ms_per_step"],
+                "kernel_us_per_step": sm["kernel_us_per_step"], "two_launch_us_per_step": sm["two_launch_us_per_step"],
+                "roofline_bound": sm["roofline"]["bound"], "roofline_frac": sm["roofline"]["frac"],
+                "roofline_achieved": sm["roofline"]["achieved"], "roofline_unit": sm["roofline"]["unit"],
+                "per_linear_frac": sm["roofline"]["per_linear_frac"],
+                "rotate_quant_frac": sm["rotate_quant"]["frac"], "rotate_quant_gbs": sm["rotate_quant"]["achieved"],
+                "plans": {n: f"{'fused ' if p['fused'] else ''}{['token-major', 'feature-major', 'gemv'][p['gemm_kind']]}"
+                             f"{' bn' + str(p['tile_n']) if p['tile_n'] else ''}{' pair' if p['cta_pair'] else ''}"
+                             f"{' stream-K' if p['stream_k'] else ''}{' split' + str(p['k_splits']) if p['k_splits'] > 1 else ''}"
+                          for n, p in sm["plans"].items()},
+                "sets": len(sreps),
+            }
+            del sreps
+            torch.cuda.empty_cache()
+        line["sub_results"] = subs
+        line["context"] = context_rows(w, reps, stream, peaks)
     if world == 1 and not args.no_cpu_baseline:
         cb = time_oracle(w, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {
@@ -540,25 +680,39 @@ def ours_arm(args, w, rank, world, local_rank):
             "sample": f"{cb['rows']} of {w.M} tokens through every linear (rotate+quant, int GEMM, dequant) "
                       f"in {cb['seconds']:.1f} s; weights converted untimed; CPU {cpu_model()}",
         }
+        single = {}
+        for name in ("tiny_w8a8", "vit_l_w8a8"):
+            c = time_oracle(workload_by_name(name), budget_s=args.cpu_budget / 4, threads=1)
+            single[name] = {"tokens_per_s": c["tokens_per_s"], "rows": c["rows"], "seconds": round(c["seconds"], 2)}
+        line["cpu_baseline"]["single_thread"] = single
     print(json.dumps(line), flush=True)
+
+
+SUB_WORKLOADS = ("vit_l_w8a8", "vit_l_w4a4", "vit_l_mixed", "msweep_w8a8_M1", "msweep_w8a8_M16",
+                 "msweep_w8a8_M128", "msweep_w8a8_M1024", "msweep_w8a8_M4096", "msweep_w8a8_M16384")
+
+
+def workload_by_name(name: str) -> wl.Workload:
+    if name.startswith("msweep"):
+        return wl.msweep(int(name.rsplit("M", 1)[1]))
+    return wl.WORKLOADS[name]
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="vit_l_w8a8")
-    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--workload", default="dit_w8a8")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub-results", action="store_true")
+    ap.add_argument("--sub-steps", type=int, default=10)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.workload.startswith("msweep"):
-        w = wl.msweep(int(args.workload.rsplit("M", 1)[1]))
-    else:
-        w = wl.WORKLOADS[args.workload]
+    w = workload_by_name(args.workload)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -182,6 +182,40 @@ convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const 
                                      void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * How convrot_linear_w8a8 / convrot_linear_w4a4 would run a call of these
+ * sizes with a workspace of workspace_bytes on the current device (no launch):
+ *   fused      1: the linear rotates and quantizes inside its GEMM kernel.
+ *              For the fewest tokens (the weight-streaming plan, block 128, K
+ *              a multiple of 512 up to 8192) every CTA rotates the few token
+ *              rows itself into shared memory while its first weights load.
+ *              For more than 128 tokens (W8A8, block 128, K <= 2048, workspace
+ *              >= convrot_linear_workspace_bytes) activation warps in the
+ *              GEMM's CTAs rotate and quantize the tokens into the workspace
+ *              beside the tensor-core main loop, which loads each 128-token
+ *              panel once all of its rows are done; a tiny kernel zeroing the
+ *              panel counters goes first.  0: the activation kernel, then the
+ *              GEMM.
+ *   launches   kernels per call.
+ *   gemm_kind  0: token-major tensor-core tiles (128 tokens x tile_n
+ *              features); 1: feature-major tiles (128 features x tile_n
+ *              tokens); 2: the weight-streaming kernel (dp4a).
+ *   cta_pair / stream_k / k_splits: CTA pairs (cta_group::2), stream-K shares,
+ *              K slices of the feature-major split.
+ * (Civarchive ConvRot release, "Future improvements": fusion of the steps.)
+ */
+typedef struct {
+    int launches;
+    int fused;
+    int gemm_kind;
+    int tile_n;
+    int cta_pair;
+    int stream_k;
+    int k_splits;
+} convrot_linear_plan_t;
+convrot_status_t convrot_linear_plan(int64_t M, int64_t K, int64_t N, int bits, int block, size_t workspace_bytes,
+                                     convrot_linear_plan_t *plan);
+
+/*
  * The two launches of convrot_linear_w8a8 / convrot_linear_w4a4, callable
  * separately (same arguments, same workspace layout): first rotate and
  * quantize X into the workspace, then run the integer GEMM + dequant from it.
@@ -198,8 +232,9 @@ convrot_status_t convrot_linear_gemm(const void *workspace, size_t workspace_byt
 
 /*
  * The integer GEMM with its dequantizing epilogue alone, on given codes (the
- * last two steps of the linear): Y[m,n] = fp16((float(acc) * x_scale[m]) *
- * w_scale[n] + bias[n]), acc = sum_k Xq[m,k] Wq[n,k].
+ * last two steps of the linear): Y[m,n] = fp16(fma(fp32(float(acc) *
+ * x_scale[m]), w_scale[n], bias[n])) -- one rounding for the product with
+ * x_scale, one for the fused multiply-add -- with acc = sum_k Xq[m,k] Wq[n,k].
  *   Xq [M x K] int8, Wq [N x K] int8 (w8a8); packed int4 [M x K/2], [N x K/2] (w4a4).
  *   acc_out  [M x N] int32 or NULL: receives acc (for exact-integer testing).
  */
@@ -238,6 +273,22 @@ convrot_status_t convrot_linear_w8a8_noalloc(const void *X, int64_t M, int64_t K
  * reported an error.
  */
 convrot_status_t convrot_device_status(void *stream);
+
+/*
+ * Diagnostics (no counterpart on the source pages): exercises the failure
+ * path of the kernels' bounded device-side waits without a fault.  Launches one
+ * tiny kernel that waits, through the same wait routines the linear's kernels
+ * use, on something that never completes -- kind 0: an mbarrier phase that no
+ * thread completes; kind 1: a fused-prologue flag word that no CTA publishes --
+ * with a limit of limit_ns nanoseconds (1 us .. 1 s).  The wait gives up, the
+ * kernel records CONVROT_ERR_TIMEOUT in the device status word (reported and
+ * cleared by the next convrot_device_status) and returns; nothing traps and the
+ * context stays usable.
+ *   result  16 bytes of device memory, 16-byte aligned: result[0] = 1 if the
+ *           wait succeeded (0 expected), result[1] = 1 if it abandoned the
+ *           wait; bytes 8..15 serve as the flag word of kind 1.
+ */
+convrot_status_t convrot_test_abandoned_wait(int kind, uint64_t limit_ns, int32_t *result, void *stream);
 
 /* Static description of a status code (never NULL). */
 const char *convrot_status_string(convrot_status_t status);

@@ -22,7 +22,8 @@
  *   - salahadawi.com, "Explanation of INT8 ConvRot", tables "8-bit INT type
  *     models": INT8 encoding, Row-wise scaling, ConvRot quantization method.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent (none of these pages fixes the
+ * block order, the signs, the clip grid or the rounding of the steps below):
  *   R      = blockdiag(R_b, ..., R_b),  R_b = H_b / sqrt(b), H_b the Sylvester
  *            Hadamard matrix in natural order, no random signs, disjoint blocks.
  *   X~     = fp32( X . R ) evaluated as a dense fp64 product per block.

@@ -25,7 +25,18 @@ EXPORTED = (
     "convrot_device_status", "convrot_status_string", "convrot_last_error", "convrot_version",
     "convrot_linear_w8a8_noalloc", "convrot_linear_quant_act", "convrot_linear_gemm",
     "convrot_linear_workspace_bytes", "convrot_tensorwise_workspace_bytes", "convrot_quantize_weight_tensorwise",
+    "convrot_test_abandoned_wait", "convrot_linear_plan",
 )
+
+
+class LinearPlan(ctypes.Structure):
+    """convrot_linear_plan_t: how a linear call runs (see include/convrot.h)."""
+    _fields_ = [("launches", ctypes.c_int), ("fused", ctypes.c_int), ("gemm_kind", ctypes.c_int),
+                ("tile_n", ctypes.c_int), ("cta_pair", ctypes.c_int), ("stream_k", ctypes.c_int),
+                ("k_splits", ctypes.c_int)]
+
+    def as_dict(self):
+        return {name: getattr(self, name) for name, _ in self._fields_}
 
 
 class ConvRotError(RuntimeError):
@@ -63,6 +74,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
             "convrot_linear_quant_act": (i32, [P, i64, i64, i32, i32, P, sz, P]),
             "convrot_linear_gemm": (i32, [P, sz, i64, i64, i32, P, P, i64, P, P, P]),
             "convrot_device_status": (i32, [P]),
+            "convrot_test_abandoned_wait": (i32, [i32, ctypes.c_uint64, P, P]),
+            "convrot_linear_plan": (i32, [i64, i64, i64, i32, i32, sz, ctypes.POINTER(LinearPlan)]),
             "convrot_status_string": (ctypes.c_char_p, [i32]),
             "convrot_last_error": (ctypes.c_char_p, []),
             "convrot_version": (i32, []),
@@ -261,6 +274,20 @@ def convrot_linear_w8a8_noalloc(X, Wq, w_scale, block, bias=None, Y=None, stream
 def convrot_device_status(stream=None):
     """Synchronizes the stream and raises if a kernel recorded a device-side timeout."""
     _check(load_library().convrot_device_status(_stream(stream)))
+
+
+def convrot_linear_plan(M: int, K: int, N: int, bits: int, block: int, workspace_bytes: int) -> dict:
+    """How a linear of these sizes runs with this workspace (launches, fused, GEMM kind, tile)."""
+    plan = LinearPlan()
+    _check(load_library().convrot_linear_plan(M, K, N, bits, block, workspace_bytes, ctypes.byref(plan)))
+    return plan.as_dict()
+
+
+def convrot_test_abandoned_wait(kind: int, limit_ns: int, result: torch.Tensor, stream=None):
+    """Diagnostics: one bounded device wait that runs out (kind 0: mbarrier,
+    1: fused-prologue flag) after limit_ns; result is an int32[4] CUDA tensor."""
+    _dev(result, "result")
+    _check(load_library().convrot_test_abandoned_wait(kind, limit_ns, _ptr(result), _stream(stream)))
 
 
 def convrot_version() -> int:

@@ -323,6 +323,7 @@ struct GemmPlan {
 
 constexpr int kMaxSplitTiles = 512;              // split-K counters in a linear's workspace
 constexpr size_t kCounterBytes = kMaxSplitTiles * 4;
+static_assert(kCounterBytes == convrot::kFuseMaxPanels * 4, "the fused linear's panel counters fill the counter area");
 constexpr int64_t kSwapMaxTokens = 128;          // feature-major up to this many tokens
 constexpr int kSwapTokens = 32;                  // token tile of the feature-major GEMM
 constexpr int64_t kMaxSplitFeatures = 32768;     // split K only for N up to this
@@ -411,20 +412,37 @@ size_t split_buffer_bytes(const GemmPlan &p, int64_t M, int64_t N) {
     return p.splits > 1 ? round256(static_cast<size_t>(M) * N * 4) : 0;
 }
 
+// The fused linear's activation input: the fp16 X, its block size and the
+// panel counters in the workspace (the codes and scales go to the GEMM's Xc / sx).
+struct FusePrologue {
+    const void *X = nullptr;
+    int log2b = 0;
+    unsigned int *panels = nullptr;
+};
+
+// Block sizes the fused linear is built for (others take two launches).
+constexpr bool fuse_block_supported(int log2b) { return log2b == 7; }
+
 // Xc: activation codes (M x K), Wc: weight codes (N x K); A4 / B4 of Cfg refer
 // to the MMA's operands (token-major: A = activations; feature-major: A = weights).
-template <class Cfg>
+// FL >= 0: fused prologue with block 2^FL and FB-wide activation codes (Xc and
+// sx are then written by the kernel).
+template <class Cfg, int FL = -1, int FB = 8>
 convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, const void *Wc, int64_t M, int64_t N,
                                  int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
                                  int32_t *acc_out, cudaStream_t st, int splits, int32_t *acc_buf,
-                                 unsigned int *counters, int streamk = 0) {
+                                 unsigned int *counters, int streamk = 0, const FusePrologue *fuse = nullptr) {
+    const auto kern = convrot::gemm_i8_tcgen05_kernel<Cfg, FL, FB>;
+    const __half *fx = fuse ? static_cast<const __half *>(fuse->X) : nullptr;
+    int8_t *fq = fuse ? static_cast<int8_t *>(const_cast<void *>(Xc)) : nullptr;
+    float *fs = fuse ? const_cast<float *>(sx) : nullptr;
+    unsigned int *ff = fuse ? fuse->panels : nullptr;
     {
         static std::mutex mu;
         static bool done[kMaxDevices] = {};
         std::lock_guard<std::mutex> lock(mu);
         if (!done[dev]) {
-            cudaError_t e = cudaFuncSetAttribute(convrot::gemm_i8_tcgen05_kernel<Cfg>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
             CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
             done[dev] = true;
         }
@@ -463,25 +481,24 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, cons
                 occ.attrs = attr;
                 occ.numAttrs = 1;
                 int n = 0;
-                cudaError_t e = cudaOccupancyMaxActiveClusters(&n, convrot::gemm_i8_tcgen05_kernel<Cfg>, &occ);
+                cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &occ);
                 CR_REQUIRE(e == cudaSuccess && n > 0, CONVROT_ERR_CUDA, "cudaOccupancyMaxActiveClusters: %s (%d)",
                            cudaGetErrorString(e), n);
                 max_clusters[dev] = n;
             }
         }
         const int64_t clusters = units < max_clusters[dev] ? units : max_clusters[dev];
-        launch_pdl_cluster(convrot::gemm_i8_tcgen05_kernel<Cfg>, dim3(static_cast<unsigned>(2 * clusters)),
-                           dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, 2u, ta, tb, ty, static_cast<int>(rows_a),
-                           static_cast<int>(rows_b), static_cast<int>(K), sx, sw, static_cast<const __half *>(bias),
-                           static_cast<__half *>(Y), acc_out, splits, acc_buf, counters, 0);
+        launch_pdl_cluster(kern, dim3(static_cast<unsigned>(2 * clusters)), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st,
+                           2u, ta, tb, ty, static_cast<int>(rows_a), static_cast<int>(rows_b), static_cast<int>(K), sx,
+                           sw, static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out, splits, acc_buf,
+                           counters, 0, fx, fq, fs, ff);
         return launch_status("gemm_i8_tcgen05 (CTA pairs)");
     }
     // persistent: one CTA per SM (stream-K: exactly the planned number of shares)
     const int grid = streamk > 0 ? streamk : static_cast<int>(units < info->sms ? units : info->sms);
-    launch_pdl(convrot::gemm_i8_tcgen05_kernel<Cfg>, dim3(grid), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, ta, tb,
-               ty, static_cast<int>(rows_a), static_cast<int>(rows_b), static_cast<int>(K), sx, sw,
-               static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out, splits, acc_buf, counters,
-               streamk);
+    launch_pdl(kern, dim3(grid), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, ta, tb, ty, static_cast<int>(rows_a),
+               static_cast<int>(rows_b), static_cast<int>(K), sx, sw, static_cast<const __half *>(bias),
+               static_cast<__half *>(Y), acc_out, splits, acc_buf, counters, streamk, fx, fq, fs, ff);
     return launch_status("gemm_i8_tcgen05");
 }
 
@@ -511,6 +528,35 @@ convrot_status_t launch_gemv(const void *Xc, const void *Wc, int64_t M, int64_t 
 }
 
 // X4 / W4: activation / weight codes packed int4.
+// The fused W8A8 linear (token-major, whole tiles, block 2^7): the plan's tile
+// width and pair choice, launched as one kernel whose activation warps rotate
+// and quantize X beside the main loop.
+convrot_status_t launch_gemm_fused(DeviceInfo *info, int dev, const void *Xc, const void *Wc, int64_t M, int64_t N,
+                                   int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
+                                   cudaStream_t st, const GemmPlan &p, const FusePrologue &fz) {
+    using convrot::GemmCfg;
+    if (p.bn == 192)
+        return launch_gemm_cfg<GemmCfg<192, false, false, false, false, false, true>, 7, 8>(
+            info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, nullptr, st, 1, nullptr, nullptr, 0, &fz);
+    if (p.bn == 256) {
+        if (p.pair)
+            return launch_gemm_cfg<GemmCfg<256, false, false, false, true, false, true>, 7, 8>(
+                info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, nullptr, st, 1, nullptr, nullptr, 0, &fz);
+        return launch_gemm_cfg<GemmCfg<256, false, false, false, false, false, true>, 7, 8>(
+            info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, nullptr, st, 1, nullptr, nullptr, 0, &fz);
+    }
+    return launch_gemm_cfg<GemmCfg<128, false, false, false, false, false, true>, 7, 8>(
+        info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, nullptr, st, 1, nullptr, nullptr, 0, &fz);
+}
+
+// K limit of the fused linear (one row fits its activation warps once).
+// K limit of the fused linear.  One row fits its activation warps once up to
+// 8192 features, but beyond 2048 a unit holds fewer than 4 rows and the eight
+// activation warps would take longer than the main loop they run beside.
+constexpr int64_t kFuseMaxK = 2048;
+static_assert(kFuseMaxK <= convrot::GemmCfg<256, false, false, false, false, false, true>::ACT_MAX_K,
+              "a row fits the activation warps");
+
 template <bool X4, bool W4>
 convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const void *Wc, int64_t M, int64_t N,
                              int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
@@ -559,6 +605,52 @@ convrot_status_t check_gemm_args(const void *Xq, const float *xs, int64_t M, con
     CR_REQUIRE(aligned(ws, 16), CONVROT_ERR_ALIGNMENT, "w_scale must be 16-byte aligned");
     CR_REQUIRE(bias == nullptr || aligned(bias, 16), CONVROT_ERR_ALIGNMENT, "bias must be 16-byte aligned");
     return ok();
+}
+
+// The fused small-M linear (rotate + quantize in every CTA, then the weight
+// stream): for the plans that take the weight-streaming GEMM, block 128 and
+// K a multiple of 512 up to 8192.
+static bool fused_gemv_plan(int sms, int64_t M, int64_t K, int64_t N, int bits, int block, GemmPlan *plan) {
+    if (!fuse_block_supported(ilog2(block)) || K % convrot::kGemvChunk != 0 || K > convrot::kGemvFusedMaxK) return false;
+    const GemmPlan p = plan_gemm(sms, M, N, K, false, bits == 4);
+    if (!p.gemv) return false;
+    *plan = p;
+    return true;
+}
+
+template <bool W4, int MT>
+convrot_status_t launch_gemv_fused_mt(int dev, int sms, const void *X, const void *Wc, int64_t M, int64_t N,
+                                      int64_t K, const float *sw, const void *bias, void *Y, int8_t *xq,
+                                      float *xs, cudaStream_t st) {
+    auto kern = convrot::gemv_fused_kernel<W4, MT, 7>;
+    {
+        static std::mutex mu;
+        static bool done[kMaxDevices] = {};
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 convrot::gemv_fused_smem_bytes(MT, convrot::kGemvFusedMaxK));
+            CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+            done[dev] = true;
+        }
+    }
+    const int64_t groups = (N + 3) / 4;
+    const int grid = static_cast<int>(groups < sms ? groups : sms);
+    launch_pdl(kern, dim3(grid), dim3(convrot::kGemvFusedThreads),
+               static_cast<size_t>(convrot::gemv_fused_smem_bytes(MT, static_cast<int>(K))), st,
+               static_cast<const __half *>(X), static_cast<const uint8_t *>(Wc), sw, static_cast<const __half *>(bias),
+               static_cast<__half *>(Y), xq, xs, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
+    return launch_status("gemv_fused");
+}
+
+template <bool W4>
+convrot_status_t launch_gemv_fused(int dev, int sms, const void *X, const void *Wc, int64_t M, int64_t N, int64_t K,
+                                   const float *sw, const void *bias, void *Y, int8_t *xq, float *xs,
+                                   cudaStream_t st) {
+    if (M <= 1) return launch_gemv_fused_mt<W4, 1>(dev, sms, X, Wc, M, N, K, sw, bias, Y, xq, xs, st);
+    if (M <= 2) return launch_gemv_fused_mt<W4, 2>(dev, sms, X, Wc, M, N, K, sw, bias, Y, xq, xs, st);
+    if (M <= 4) return launch_gemv_fused_mt<W4, 4>(dev, sms, X, Wc, M, N, K, sw, bias, Y, xq, xs, st);
+    return launch_gemv_fused_mt<W4, 8>(dev, sms, X, Wc, M, N, K, sw, bias, Y, xq, xs, st);
 }
 
 }  // namespace
@@ -764,6 +856,32 @@ static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int
                                  static_cast<int64_t>(zero_bytes / 16));
 }
 
+// The GEMM plan of a linear's second launch: split K only when the workspace
+// holds the counters and the sum buffer (which the activation half zeroed).
+static GemmPlan two_launch_plan(int sms, int64_t M, int64_t N, int64_t K, int bits, size_t workspace_bytes) {
+    GemmPlan p = plan_gemm(sms, M, N, K, true, bits == 4);
+    const size_t base = convrot_workspace_bytes(M, K, bits) + kCounterBytes;
+    if ((p.splits > 1 || p.streamk > 0) && workspace_bytes < base + split_buffer_bytes(p, M, N))
+        p = plan_gemm(sms, M, N, K, false, bits == 4);
+    return p;
+}
+
+// Whether a linear runs as one fused launch (token-major tiles for more than
+// 128 tokens, a block size the prologue is built for, K within its consumer
+// warps' reach and a workspace with room for the per-CTA flag words, which
+// live in the split-K counter area that this plan does not use), and its plan.
+static bool fused_plan(int sms, int64_t M, int64_t K, int64_t N, int bits, int block, size_t workspace_bytes,
+                       GemmPlan *plan) {
+    if (M <= kSwapMaxTokens || !fuse_block_supported(ilog2(block)) || K > kFuseMaxK) return false;
+    if (bits != 8) return false;
+    if ((M + 127) / 128 > convrot::kFuseMaxPanels) return false;
+    if (workspace_bytes < convrot_workspace_bytes(M, K, bits) + kCounterBytes) return false;
+    const GemmPlan p = plan_gemm(sms, M, N, K, false, bits == 4);  // whole tiles: no split state
+    if (p.swap || p.gemv) return false;
+    *plan = p;
+    return true;
+}
+
 static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace_bytes, int64_t M, int64_t K,
                                          int bits, const void *Wq, const float *w_scale, int64_t N,
                                          const void *bias, void *Y, cudaStream_t st) {
@@ -777,17 +895,56 @@ static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace
     int dev;
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
-    // split K only when the workspace holds the counters and the sum buffer
-    // (which the activation half zeroed)
-    GemmPlan p = plan_gemm(info->sms, M, N, K, true, bits == 4);
-    const size_t base = convrot_workspace_bytes(M, K, bits) + kCounterBytes;
-    if ((p.splits > 1 || p.streamk > 0) && workspace_bytes < base + split_buffer_bytes(p, M, N))
-        p = plan_gemm(info->sms, M, N, K, false, bits == 4);
+    const GemmPlan p = two_launch_plan(info->sms, M, N, K, bits, workspace_bytes);
     if (bits == 8)
         return launch_gemm<false, false>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st, p, acc_buf,
                                          counters);
     return launch_gemm<false, true>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st, p, acc_buf,
                                     counters);
+}
+
+// One launch for the whole linear where the fused prologue applies (see
+// fused_plan).  *fused tells whether it ran.
+static convrot_status_t linear_fused_impl(int bits, const void *X, int64_t M, int64_t K, const void *Wq,
+                                          const float *w_scale, int64_t N, const void *bias, int block, void *Y,
+                                          void *workspace, size_t workspace_bytes, cudaStream_t st, bool *fused) {
+    *fused = false;
+    if (workspace == nullptr) return ok();
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    GemmPlan p;
+    if (fused_gemv_plan(info->sms, M, K, N, bits, block, &p)) {
+        void *xq;
+        float *xs;
+        workspace_parts(workspace, M, K, &xq, &xs);
+        CR_TRY(check_gemm_args(xq, xs, M, Wq, w_scale, N, K, bias, Y));
+        *fused = true;
+        if (bits == 8)
+            return launch_gemv_fused<false>(dev, info->sms, X, Wq, M, N, K, w_scale, bias, Y,
+                                            static_cast<int8_t *>(xq), xs, st);
+        return launch_gemv_fused<true>(dev, info->sms, X, Wq, M, N, K, w_scale, bias, Y, static_cast<int8_t *>(xq),
+                                       xs, st);
+    }
+    if (!fused_plan(info->sms, M, K, N, bits, block, workspace_bytes, &p)) return ok();
+    const int log2b = ilog2(block);
+    CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
+    CR_REQUIRE(aligned(workspace, 16), CONVROT_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+    void *xq;
+    float *xs;
+    unsigned int *counters;
+    workspace_parts(workspace, M, K, &xq, &xs, &counters);
+    CR_TRY(check_gemm_args(xq, xs, M, Wq, w_scale, N, K, bias, Y));
+    FusePrologue fz;
+    fz.X = X;
+    fz.log2b = log2b;
+    fz.panels = counters;
+    *fused = true;
+    // zero the panel counters (programmatic launch: overlaps the previous kernel's tail)
+    const int panels = static_cast<int>((M + 127) / 128);
+    launch_pdl(convrot::fuse_zero_kernel, dim3(1), dim3(256), 0, st, counters, panels);
+    CR_TRY(launch_status("fuse_zero"));
+    return launch_gemm_fused(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, st, p, fz);
 }
 
 static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t K, const void *Wq,
@@ -797,7 +954,12 @@ static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t 
     CR_TRY(check_linear_shape(M, K, block, bits, N));
     if (M == 0 || N == 0) return ok();
     CR_REQUIRE(X && Wq && w_scale && Y, CONVROT_ERR_INVALID_ARG, "null pointer argument");
+    CR_TRY(check_workspace(workspace, workspace_bytes, M, K, bits));
+    CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    bool fused = false;
+    CR_TRY(linear_fused_impl(bits, X, M, K, Wq, w_scale, N, bias, block, Y, workspace, workspace_bytes, st, &fused));
+    if (fused) return ok();
     CR_TRY(linear_act_impl(X, M, K, block, bits, workspace, workspace_bytes, st, N));
     return linear_gemm_impl(workspace, workspace_bytes, M, K, bits, Wq, w_scale, N, bias, Y, st);
 }
@@ -907,6 +1069,46 @@ convrot_status_t convrot_linear_w8a8_noalloc(const void *X, int64_t M, int64_t K
         scratch = g_noalloc_ptr[dev];
     }
     return linear_impl(8, X, M, K, Wq, w_scale, N, bias, block, Y, scratch, kNoAllocScratchBytes, stream);
+}
+
+convrot_status_t convrot_linear_plan(int64_t M, int64_t K, int64_t N, int bits, int block, size_t workspace_bytes,
+                                     convrot_linear_plan_t *plan) {
+    g_last_error.clear();
+    CR_TRY(check_linear_shape(M, K, block, bits, N));
+    CR_REQUIRE(plan != nullptr, CONVROT_ERR_INVALID_ARG, "null pointer argument");
+    *plan = convrot_linear_plan_t();
+    if (M == 0 || N == 0) return ok();
+    CR_REQUIRE(workspace_bytes >= convrot_workspace_bytes(M, K, bits), CONVROT_ERR_WORKSPACE,
+               "workspace of %zu bytes given, %zu needed", workspace_bytes, convrot_workspace_bytes(M, K, bits));
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    GemmPlan p;
+    const bool fused_gemv = fused_gemv_plan(info->sms, M, K, N, bits, block, &p);
+    const bool fused = fused_gemv || fused_plan(info->sms, M, K, N, bits, block, workspace_bytes, &p);
+    if (!fused) p = two_launch_plan(info->sms, M, N, K, bits, workspace_bytes);
+    // counter zeroing + fused GEMM, one fused weight-streaming kernel, or activation kernel + GEMM
+    plan->launches = fused_gemv ? 1 : 2;
+    plan->fused = fused ? 1 : 0;
+    plan->gemm_kind = p.gemv ? 2 : (p.swap ? 1 : 0);
+    plan->tile_n = p.gemv ? 0 : p.bn;
+    plan->cta_pair = p.pair ? 1 : 0;
+    plan->stream_k = p.streamk > 0 ? 1 : 0;
+    plan->k_splits = p.splits;
+    return ok();
+}
+
+convrot_status_t convrot_test_abandoned_wait(int kind, uint64_t limit_ns, int32_t *result, void *stream) {
+    g_last_error.clear();
+    CR_REQUIRE(kind == 0 || kind == 1, CONVROT_ERR_INVALID_ARG, "kind = %d must be 0 or 1", kind);
+    CR_REQUIRE(limit_ns >= 1000 && limit_ns <= 1000000000ull, CONVROT_ERR_INVALID_ARG,
+               "limit_ns = %llu must be in [1 us, 1 s]", static_cast<unsigned long long>(limit_ns));
+    CR_REQUIRE(result != nullptr && aligned(result, 16), CONVROT_ERR_ALIGNMENT, "result must be 16-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    convrot::abandoned_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(kind, limit_ns, result);
+    return launch_status("abandoned_wait");
 }
 
 convrot_status_t convrot_device_status(void *stream) {

@@ -62,13 +62,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Waits until the phase with the given parity has completed.  Returns false
 // (and records the timeout in the status word and in *abort) if that takes
-// longer than kWaitLimitNs or if another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// longer than limit_ns or if another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             atomicOr(&g_device_status, kStatusTimeout);
             *abort = 1;
             return false;
@@ -101,7 +102,40 @@ __device__ __forceinline__ void flag_raise(unsigned int *flag) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(1u) : "memory");
 }
 
+// Bounded wait taken by every lane of a warp: true only if it succeeded for
+// all of them, so that a timeout leaves the warp converged (the callers then
+// use warp-collective instructions).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
+// Bounded wait used while draining: ignores the abort flag, still time-limited.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
+    int dummy = 0;
+    mbar_wait(bar, parity, &dummy);
+}
+
+// Barrier `id` (1..15) over `nthreads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------- TMA
+
+// 1-D bulk copy global -> shared of `bytes` contiguous bytes (a multiple of 16;
+// both addresses 16-byte aligned), completing on `bar`.  No multicast.
+__device__ __forceinline__ void bulk_load_1d(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+// Orders this thread's generic-proxy global accesses with later (or, on the
+// writing side, other threads' later) async-proxy accesses such as TMA loads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

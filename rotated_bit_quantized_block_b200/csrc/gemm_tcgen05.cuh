@@ -2,7 +2,7 @@
 // ConvRot linear, on sm_100a 5th-generation tensor cores.
 //
 //   acc[m,n] = sum_k qx[m,k] * qw[n,k]                      (tcgen05.mma kind::i8, int32 in TMEM)
-//   Y[m,n]   = fp16( (float(acc) * s_x[m]) * s_w[n] + bias[n] )   (fused epilogue)
+//   Y[m,n]   = fp16( fma( fp32(float(acc) * s_x[m]), s_w[n], bias[n] ) )   (fused epilogue)
 //
 // Method: civarchive.com "SAM 3.1 Multiplex ConvRot" release, "Quantization
 // recipe" (W8A8 / W4A4 operations, per-row scales; INT4 multiplication falls
@@ -33,9 +33,25 @@
 //     across CTAs: every slice adds its int32 partial into a zeroed M x N
 //     buffer (red.add), and the slice that counts in last dequantizes the sum
 //     and zeroes the buffer again.
+//
+// Fused linear (Cfg::FUSE, token-major): the kernel also rotates and
+// quantizes the activations.  ACT_WARPS extra warps per CTA (register-fed, no
+// shared memory) work through "units" of rows -- unit u (RPR = 32*ACT_WARPS /
+// (K/32) rows) belongs to CTA u mod grid, so the first units of every CTA
+// cover the first 128-token panels -- writing codes and per-token scales into
+// the workspace (left in L2) and counting each finished unit into the counter
+// of every panel it touches.  The producer loads a panel's A tiles only once
+// its counter shows all of the panel's units (acquire, bounded wait), and
+// issues the stage's weight tile first so that it is in flight meanwhile; the
+// epilogue re-acquires the counter before it reads the panel's scales.  The
+// rotation thus runs beside the main loop instead of in a launch of its own,
+// and every panel is rotated exactly once.  The counters are zeroed by a small
+// kernel launched just before (programmatic dependency).  The grid is at most
+// one CTA (or CTA pair) per SM, all co-resident.
 #pragma once
 
 #include "device_utils.cuh"
+#include "rotate_quant.cuh"
 
 namespace convrot {
 
@@ -50,7 +66,8 @@ constexpr int kStreamKFlags = 256;
 // PAIR: a cluster of two CTAs shares each 256 x BN tile through one
 // cta_group::2 MMA (each CTA loads and keeps 128 rows of A and BN/2 rows of B).
 // SK: token-major stream-K (equal shares of all tiles' K steps per CTA).
-template <int BN_, bool A4_, bool B4_, bool SWAP_ = false, bool PAIR_ = false, bool SK_ = false>
+// FUSE: token-major linear with ACT_WARPS activation warps (see the header).
+template <int BN_, bool A4_, bool B4_, bool SWAP_ = false, bool PAIR_ = false, bool SK_ = false, bool FUSE_ = false>
 struct GemmCfg {
     static constexpr int BM = 128;   // rows of A per CTA
     static constexpr int BN = BN_;   // accumulator columns
@@ -60,6 +77,7 @@ struct GemmCfg {
     static constexpr bool SWAP = SWAP_;
     static constexpr bool PAIR = PAIR_;
     static constexpr bool SK = SK_;
+    static constexpr bool FUSE = FUSE_;
     static constexpr int CTAS = PAIR ? 2 : 1;      // CTAs per tile
     static constexpr int TILE_M = BM * CTAS;       // accumulator rows per tile
     static constexpr int B_ROWS = BN / CTAS;       // rows of B held by one CTA
@@ -83,7 +101,7 @@ struct GemmCfg {
     static constexpr int TMEM_COLS = 2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512));
     // epilogue warps: per TMEM lane quarter, EPI_WARPS / 4 warps split the columns
     // (token-major: four, so that enough warps hide the dequant's latencies)
-    static constexpr int EPI_WARPS = (SWAP || W4 || BN % 128 != 0) ? 8 : 16;
+    static constexpr int EPI_WARPS = (SWAP || W4 || FUSE || BN % 128 != 0) ? 8 : 16;
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // accumulator columns per epilogue warp
     // token-major: 32-column chunks (one TMEM load, one 32 x 32 fp16 output box);
     // feature-major: 16- or 32-column TMEM loads, stored directly
@@ -92,19 +110,26 @@ struct GemmCfg {
     static constexpr int OUT_BYTES = SWAP ? 0 : EPI_WARPS * OUT_BOX_BYTES;
     static constexpr int SCALE_BYTES = BN * 4 + BN * 2;  // the tile's column scale (fp32) and bias (fp16)
     static constexpr int FIRST_CONV_WARP = 2 + EPI_WARPS;
-    static constexpr int NUM_THREADS = 32 * (FIRST_CONV_WARP + CONV_WARPS);
+    // fused linear: activation warps after the converters
+    static constexpr int ACT_WARPS = FUSE ? 8 : 0;
+    static constexpr int ACT_THREADS = 32 * ACT_WARPS;
+    static constexpr int FIRST_ACT_WARP = FIRST_CONV_WARP + CONV_WARPS;
+    static constexpr int ACT_MAX_K = ACT_THREADS * kElemsPerThread;  // a row fits the activation warps once
+    static constexpr int ACT_SMEM_BYTES = FUSE ? 2 * (ACT_THREADS / 4) * 4 : 0;  // row-segment maxima, 2 units
+    static constexpr int NUM_THREADS = 32 * (FIRST_ACT_WARP + ACT_WARPS);
     static constexpr int FIXED_BARRIERS = 2 * PSTAGES + 4 + 1 + 2 + 2;
     // MMA ring depth: as many stages as fit in the shared-memory budget (at most 12)
     static constexpr int SMEM_LIMIT = 232448;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - PSTAGES * PSTAGE_BYTES - OUT_BYTES - SCALE_BYTES -
-                                       FIXED_BARRIERS * 8 - 16) /
+                                       ACT_SMEM_BYTES - FIXED_BARRIERS * 8 - 16) /
                                       (STAGE_BYTES + 16);
     static constexpr int STAGES = STAGES_FIT < 12 ? STAGES_FIT : 12;
     static constexpr int NUM_BARRIERS = 2 * STAGES + FIXED_BARRIERS;
     static constexpr int SMEM_BYTES = 1024 /* alignment slack */ + STAGES * STAGE_BYTES + PSTAGES * PSTAGE_BYTES +
-                                      OUT_BYTES + SCALE_BYTES + NUM_BARRIERS * 8 + 16;
+                                      OUT_BYTES + SCALE_BYTES + ACT_SMEM_BYTES + NUM_BARRIERS * 8 + 16;
     static constexpr uint32_t IDESC = idesc_i8(TILE_M, BN);
     static_assert(STAGES >= 2, "pipeline depth");
+    static_assert(!FUSE || (!SWAP && !A4 && !SK), "fused linear: token-major, int8 activation codes, whole tiles");
     static_assert(!PAIR || (!SWAP && !A4 && !B4 && BN == 256), "CTA pairs: token-major W8A8, 256-wide tiles");
     static_assert(!SK || (!SWAP && !PAIR), "stream-K: token-major, single CTAs");
     static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
@@ -113,19 +138,6 @@ struct GemmCfg {
     static_assert(TMEM_COLS >= 2 * BN, "accumulators fit the allocation");
     static_assert(EPI_COLS % CHUNK == 0, "epilogue chunking");
 };
-
-// Bounded wait taken by every lane of a warp: true only if it succeeded for
-// all of them, so that a timeout leaves the warp converged (the callers then
-// use warp-collective instructions).
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
-}
-
-// Bounded wait used while draining: ignores the abort flag, still time-limited.
-__device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
-    int dummy = 0;
-    mbar_wait(bar, parity, &dummy);
-}
 
 // Sign-extends 16 packed int4 codes (8 bytes, low nibble = even element) to 16
 // bytes holding 16 * code: shifting each nibble into the high half of its byte
@@ -174,6 +186,153 @@ __device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[CHUN
     else tmem_ld_32x16(taddr, r);
 }
 
+// ---------------------------------------------------------------- fused linear: panel counters
+//
+// One 32-bit counter per 128-token panel, in the workspace's counter area:
+// the number of finished activation units that touch the panel.  A small
+// kernel launched just before the fused kernel zeroes them (the fused kernel
+// waits for it through its programmatic-launch dependency), so every launch,
+// CUDA-graph replays included, counts from zero whatever the area held before.
+constexpr int kFuseMaxPanels = 512;  // counters in the 2 KB area
+
+// Zeroes the n panel counters of the next fused launch (one block).
+__global__ void __launch_bounds__(256) fuse_zero_kernel(unsigned int *counters, int n) {
+    pdl_wait();  // the previous launch on this workspace may still count into them
+    for (int i = threadIdx.x; i < n; i += blockDim.x) counters[i] = 0u;
+    pdl_launch_dependents();
+}
+
+// Rows per activation unit of `nt` threads (L = K/32 threads per row).
+__host__ __device__ __forceinline__ int fuse_unit_rows(int nt, int K) { return nt / (K / kElemsPerThread); }
+
+// Number of units that touch panel p (rows [128 p, min(128 p + 128, M))).
+__device__ __forceinline__ uint32_t fuse_panel_units(int64_t M, int rpr, int64_t p) {
+    const int64_t r0 = 128 * p;
+    const int64_t r1 = (r0 + 128 < M ? r0 + 128 : M) - 1;
+    return static_cast<uint32_t>(r1 / rpr - r0 / rpr + 1);
+}
+
+// Waits (acquire, bounded) until panel p's counter shows all of its units.
+__device__ __forceinline__ bool fuse_panel_wait(const unsigned int *counters, int64_t M, int rpr, int64_t p,
+                                                volatile int *abort, uint64_t limit_ns = kWaitLimitNs) {
+    const unsigned int want = fuse_panel_units(M, rpr, p);
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counters + p) : "memory");
+        if (v == want) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            atomicOr(&g_device_status, kStatusTimeout);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+// The activation warps of one CTA (thread at = 0 .. NT-1): rotate and quantize
+// units blockIdx.x, blockIdx.x + gridDim.x, ... into Xq / x_scale (codes one
+// byte each, range of BITS), loading the next unit while the current one is
+// worked on, and count each finished unit into the counters of the panels it
+// touches (release: the consumers acquire the counter, then fence the async
+// proxy before their TMA loads).  Rows spanning several warps meet in s_part
+// behind named barrier bar_id (all NT threads join it the same number of times).
+template <int LOG2B, int BITS, int NT>
+__device__ __forceinline__ void fuse_act_worker(int at, const __half *__restrict__ X, int64_t M, int K,
+                                                int8_t *Xq, float *x_scale, unsigned int *counters,
+                                                float *s_part, int bar_id) {
+    const int lane = at & 31;
+    const int L = K / kElemsPerThread;
+    const int rpr = NT / L;
+    const int r = at / L, l = at - r * L;
+    const int g = l >> 2, p = l & 3;
+    const int elem0 = 128 * g + 8 * p;
+    const int G = reduce_width(L);
+    const int segs = L / G;
+    const int64_t units = (M + rpr - 1) / rpr;
+    auto load = [&](int64_t u, uint4 (&dst)[4]) {
+        const int64_t row = u * rpr + r;
+        if (r < rpr && row < M) {
+            const __half *src = X + row * K + elem0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = ld_stream_v4(src + 32 * j);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(0, 0, 0, 0);
+        }
+    };
+    uint4 raw[4];
+    int64_t u = blockIdx.x;
+    if (u < units) load(u, raw);
+    for (int it = 0; u < units; u += gridDim.x, ++it) {
+        uint4 nxt[4];
+        if (u + gridDim.x < units) load(u + gridDim.x, nxt);
+        float2 v[2][8];
+        raw_to_v(raw, v);
+        fwht_act_order<LOG2B>(v, lane);
+        float amax = 0.0f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = absmax3(amax, v[h][e].x, v[h][e].y);
+        for (int mm = 1; mm < G; mm <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, mm));
+        if (G < L) {
+            float *part = s_part + (it & 1) * (NT / 4);
+            if (r < rpr && (l & (G - 1)) == 0) part[r * segs + l / G] = amax;
+            named_bar_sync(bar_id, NT);
+            if (r < rpr) {
+                amax = part[r * segs];
+                for (int sg = 1; sg < segs; ++sg) amax = fmaxf(amax, part[r * segs + sg]);
+            }
+        }
+        const int64_t row = u * rpr + r;
+        if (r < rpr && row < M) {
+            float fac1;
+            const float sc = act_row_scale<LOG2B, BITS>(amax, &fac1);
+            if (l == 0) x_scale[row] = sc;
+            const float2 fac = f2(fac1);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[h][e] = __ffma2_rn(v[h][e], fac, f2(kRoundMagic));
+            store_codes<8>(Xq + row * K, elem0, v);
+        }
+        named_bar_sync(bar_id, NT);  // every code and scale of the unit is written
+        if (at == 0) {
+            __threadfence();
+            const int64_t r0 = u * rpr, r1 = (r0 + rpr < M ? r0 + rpr : M) - 1;
+            for (int64_t pn = r0 / 128; pn <= r1 / 128; ++pn) atomicAdd(counters + pn, 1u);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) raw[j] = nxt[j];
+    }
+}
+
+// Diagnostics: one bounded wait whose target never completes, through the
+// same routines the GEMM uses (kind 0: an mbarrier phase nobody completes;
+// kind 1: a fused linear's panel counter nobody counts into).  result[0] = 1
+// if the wait succeeded (it must not), result[1] = the abort flag it left; the
+// panel counter is result[2], cleared here first.
+__global__ void abandoned_wait_kernel(int kind, uint64_t limit_ns, int32_t *result) {
+    __shared__ uint64_t bar;
+    __shared__ int abort;
+    unsigned int *word = reinterpret_cast<unsigned int *>(result + 2);
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort = 0;
+        *word = 0;
+        fence_mbarrier_init();
+        __threadfence();
+    }
+    __syncthreads();
+    if (threadIdx.x != 0) return;
+    bool ok;
+    if (kind == 0) ok = mbar_wait(&bar, 0, &abort, limit_ns);
+    else ok = fuse_panel_wait(word, 128, 1, 0, &abort, limit_ns);
+    result[0] = ok ? 1 : 0;
+    result[1] = abort;
+}
+
 // Kernel arguments, in the MMA's terms: the accumulator is M x N (rows of A x
 // rows of B).  Token-major: M = tokens, N = output features.  Feature-major:
 // M = output features, N = tokens.  sx is always the per-token scale, sw the
@@ -182,13 +341,19 @@ __device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[CHUN
 // per-tile counters; with streamk (Cfg::SK) the partial-tile slots (TILE_M x BN
 // int32 per CTA boundary) and per-boundary arrival counts (counters[b]) and
 // ready flags (counters[kStreamKFlags + b]).
-template <class Cfg>
+// Fused linear (Cfg::FUSE; block 2^FLOG2B, activation codes one byte each in
+// the range of FBITS): X is the fp16 input, qx_out / sx_out the workspace that
+// tmA and sx cover, panels the zeroed panel counters (see above).
+template <class Cfg, int FLOG2B = -1, int FBITS = 8>
 __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                           const __grid_constant__ CUtensorMap tmY, int M, int N, int K, const float *__restrict__ sx,
+                           const __grid_constant__ CUtensorMap tmY, int M, int N, int K, const float *sx,
                            const float *__restrict__ sw, const __half *__restrict__ bias, __half *__restrict__ Y,
                            int32_t *__restrict__ acc_out, int splits, int32_t *__restrict__ acc_buf,
-                           unsigned int *__restrict__ counters, int streamk) {
+                           unsigned int *__restrict__ counters, int streamk, const __half *__restrict__ X,
+                           int8_t *qx_out, float *sx_out, unsigned int *panels) {
+    constexpr bool FUSED = Cfg::FUSE;
+    static_assert(FUSED == (FLOG2B >= 0), "the activation warps need the block size");
     constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, PSTAGES = Cfg::PSTAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -197,7 +362,8 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     uint8_t *outbuf = pring + PSTAGES * Cfg::PSTAGE_BYTES;         // per epilogue warp: 32 x 32 fp16 box
     float *col_s = reinterpret_cast<float *>(outbuf + Cfg::OUT_BYTES);         // [BN] tile column scale
     __half *bias_s = reinterpret_cast<__half *>(col_s + BN);                    // [BN] tile bias (token-major)
-    uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + Cfg::OUT_BYTES + Cfg::SCALE_BYTES);
+    float *act_part = reinterpret_cast<float *>(outbuf + Cfg::OUT_BYTES + Cfg::SCALE_BYTES);  // activation warps
+    uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + Cfg::OUT_BYTES + Cfg::SCALE_BYTES + Cfg::ACT_SMEM_BYTES);
     uint64_t *full = bars;                                         // MMA ring: operands ready
     uint64_t *empty = full + STAGES;                               // MMA ring: slot consumed
     uint64_t *pfull = empty + STAGES;                              // packed ring: TMA landed
@@ -301,6 +467,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
     pdl_wait();  // the codes, scales and split-K buffers may come from the previous kernel
     pdl_launch_dependents();
+    [[maybe_unused]] const int act_rpr = FUSED ? fuse_unit_rows(Cfg::ACT_THREADS, K) : 1;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -315,6 +482,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             for (int i = 0; i < STAGES; ++i) filled[i] = false;
             for (int i = 0; i < PSTAGES; ++i) pfilled[i] = false;
             bool ok = true;
+            [[maybe_unused]] int ready_tm = -1;  // fused: the last panel seen complete
             for (Seg g = seg_first(); ok && g.tile >= 0; g = seg_next(g)) {
                 const int tile = g.tile;
                 const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
@@ -329,14 +497,39 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                             // both CTAs' bytes land on the even CTA's barrier
                             if (leader) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
                             const uint32_t bar = cluster_addr(&full[s], 0);
-                            tma_load_2d_pair(dst, &tmA, bar, kb * Cfg::BK, tm * Cfg::TILE_M + rank * BM);
                             tma_load_2d_pair(dst + Cfg::A_BYTES, &tmB, bar, kb * Cfg::BK,
                                              tn * BN + rank * Cfg::B_ROWS);
+                            if constexpr (FUSED) {
+                                // this CTA's 128 rows of the pair's tile are panel 2 tm + rank
+                                if (tm != ready_tm) {
+                                    const int64_t pn = 2 * static_cast<int64_t>(tm) + rank;
+                                    if (pn * 128 >= M || fuse_panel_wait(panels, M, act_rpr, pn, abort)) {
+                                        fence_proxy_async_global();
+                                        ready_tm = tm;
+                                    } else {
+                                        ok = false;
+                                    }
+                                }
+                            }
+                            tma_load_2d_pair(dst, &tmA, bar, kb * Cfg::BK, tm * Cfg::TILE_M + rank * BM);
                         } else {
                             mbar_arrive_expect_tx(&full[s],
                                                   (Cfg::A4 ? 0 : Cfg::A_BYTES) + (Cfg::B4 ? 0 : Cfg::B_BYTES));
-                            if (!Cfg::A4) tma_load_2d(dst, &tmA, &full[s], kb * Cfg::BK, tm * BM);
                             if (!Cfg::B4) tma_load_2d(dst + Cfg::A_BYTES, &tmB, &full[s], kb * Cfg::BK, tn * BN);
+                            if constexpr (FUSED) {
+                                // the panel's codes: wait for its units (the weight tile is already on
+                                // its way).  After a timeout the A tile is still loaded, so that the
+                                // stage completes and drains; the launch is abandoned anyway.
+                                if (tm != ready_tm) {
+                                    if (fuse_panel_wait(panels, M, act_rpr, tm, abort)) {
+                                        fence_proxy_async_global();  // the codes were written through the generic proxy
+                                        ready_tm = tm;
+                                    } else {
+                                        ok = false;
+                                    }
+                                }
+                            }
+                            if (!Cfg::A4) tma_load_2d(dst, &tmA, &full[s], kb * Cfg::BK, tm * BM);
                         }
                         filled[s] = true;
                         last_parity[s] = ph;
@@ -344,6 +537,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                             s = 0;
                             ph ^= 1;
                         }
+                        if (!ok) break;
                     }
                     if (Cfg::W4) {
                         if (!mbar_wait(&pempty[ps], pph ^ 1, abort)) {
@@ -462,6 +656,18 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             const int tile = g.tile;
             const int acc = local & 1;
             const uint32_t acc_ph = (local >> 1) & 1;
+            const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
+            const int row0 = tm * Cfg::TILE_M + static_cast<int>(rank) * BM + q * 32;
+            const int row = row0 + lane;
+            const bool row_ok = row < M;
+            if constexpr (FUSED) {
+                // the scales of these rows: their panel's word (acquired while the tile's main loop still runs)
+                int rdy = 1;
+                if (lane == 0 && row0 < M) rdy = fuse_panel_wait(panels, M, act_rpr, row0 / 128, abort);
+                if (!__shfl_sync(0xffffffffu, rdy, 0)) break;
+            }
+            // token-major: the row's per-token scale (L2: possibly written by this launch)
+            const float sxm = (!Cfg::SWAP && row_ok) ? __ldcg(sx + row) : 0.0f;
             if (!mbar_wait_warp(&tmem_full[acc], acc_ph, abort)) break;
             tc_fence_after_sync();
             // every epilogue thread is done with the previous segment's scales
@@ -476,10 +682,6 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                 const Seg gn = seg_next(g);
                 load_scales(gn.tile >= 0 ? gn.tile : num_tiles, next_w, next_b);
             }
-            const int tm = tile / tiles_n, tn = tile - tm * tiles_n;
-            const int row0 = tm * Cfg::TILE_M + static_cast<int>(rank) * BM + q * 32;
-            const int row = row0 + lane;
-            const bool row_ok = row < M;
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
             constexpr int CH = Cfg::CHUNK;
             constexpr int NCHUNK = Cfg::EPI_COLS / CH;
@@ -517,7 +719,6 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     sk_part = acc_buf + static_cast<int64_t>(slot) * (Cfg::TILE_M * BN) + ew * (NCHUNK * 1024);
                 }
                 uint8_t *box = outbuf + ew * Cfg::OUT_BOX_BYTES;
-                const float sxm = row_ok ? sx[row] : 0.0f;
                 // 64-byte rows, 16-byte chunk g stored at g ^ ((row / 2) & 3) (64B swizzle)
                 uint8_t *brow = box + lane * 64;
                 const int xr = ((lane >> 1) & 3) << 4;
@@ -668,7 +869,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             mbar_arrive(scale_free);
         }
         if (!Cfg::SWAP && lane == 0) bulk_wait_group_all();
-    } else if (Cfg::W4) {
+    } else if (Cfg::W4 && warp < Cfg::FIRST_ACT_WARP) {
         // ------------------------------------------------------------ int4 -> int8 converters
         const int ct = threadIdx.x - 32 * Cfg::FIRST_CONV_WARP;  // 0 .. CONV_THREADS-1
         int ps = 0, us = 0;
@@ -704,6 +905,14 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                     uph ^= 1;
                 }
             }
+        }
+    }
+
+    if constexpr (FUSED) {
+        if (warp >= Cfg::FIRST_ACT_WARP) {
+            // ------------------------------------------------------------ activation warps
+            fuse_act_worker<FLOG2B < 0 ? 0 : FLOG2B, FBITS, Cfg::ACT_THREADS>(
+                threadIdx.x - 32 * Cfg::FIRST_ACT_WARP, X, M, K, qx_out, sx_out, panels, act_part, 1);
         }
     }
 

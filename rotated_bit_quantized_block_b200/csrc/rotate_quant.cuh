@@ -206,10 +206,8 @@ __host__ __device__ __forceinline__ int reduce_width(int L) {
 // ---------------------------------------------------------------------------
 // Online activation path: X (fp16, M x K) -> codes + per-token scales.
 //
-// One CTA handles `rows` consecutive rows with L = K/32 threads each (the
-// block is padded to a multiple of 32 threads; padding threads only join the
-// barriers).  Every thread issues its four 16-byte loads up front.  A thread
-// owns 32 elements of a 128-element group in two layouts:
+// A row of K elements is handled by L = K/32 threads, each owning 32 elements
+// of a 128-element group in two register layouts:
 //   layout A: element 8p + 32j + e (chunks j = 0..3 of 8 e; p = thread in the
 //             group), packed as float2 (e, e+1): butterflies on bits 1, 2, 5, 6;
 //   layout B: element 32p + i (i = 0..31 contiguous), packed as float2
@@ -219,6 +217,9 @@ __host__ __device__ __forceinline__ int reduce_width(int L) {
 // group, so every butterfly runs on the packed fp32x2 pipe and each thread
 // ends with 32 contiguous codes (16-byte stores).  The 1/sqrt(b) factor is
 // folded into the per-row code factor (exact when b is a power of 4).
+//
+// The fused linear's activation warps (end of this section) run the same
+// stages in another register layout.
 // ---------------------------------------------------------------------------
 constexpr int kXposeGroupBytes = 33 * 16;  // 32 16-byte units + 1 unit of padding
 
@@ -236,49 +237,18 @@ __device__ __forceinline__ float absmax3(float m, float x, float y) {
     return fmaxf(m, fmaxf(fabsf(x), fabsf(y)));
 }
 
-// Dynamic shared memory of the activation kernel for a block of `threads`.
+// Dynamic shared memory of the register-fed activation kernel for a block of `threads`.
 __host__ __device__ constexpr int act_smem_bytes(int threads) { return (threads / 4) * kXposeGroupBytes; }
 
-// BITS fixes the code range (8: [-127, 127], 4: [-8, 7]); PACKED stores int4
-// codes two per byte, otherwise every code takes one byte.
-template <int LOG2B, int BITS, bool PACKED>
-__global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__restrict__ X, int64_t M, int K,
-                                                                int rows, void *__restrict__ Xq,
-                                                                float *__restrict__ x_scale,
-                                                                uint4 *__restrict__ zero16,
-                                                                int64_t n_zero16) {
-    extern __shared__ __align__(16) uint8_t act_smem[];
-    __shared__ unsigned int s_amax[kMaxRowsPerCta];
-    __shared__ float s_fac[kMaxRowsPerCta];
-    const int L = K / kElemsPerThread;
-    const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int r = tid / L;
-    const int l = tid - r * L;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * rows + r;
-    const bool active = (r < rows) && (row < M);
-    const int g = l >> 2, p = l & 3;
-    constexpr float qmax = BITS == 8 ? 127.0f : 7.0f;
-    uint8_t *xbuf = act_smem + (tid >> 2) * kXposeGroupBytes;
-
-    pdl_wait();  // X may come from, and Xq may still be read by, the previous kernel
-    pdl_launch_dependents();
-    // ---- layout A: a[j][k] = (x[8p + 32j + 2k], x[8p + 32j + 2k + 1]) of group g
-    uint4 raw[4];
-    if (active) {
-        const __half *src = X + row * K + 128 * g + 8 * p;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) raw[j] = ld_stream_v4(src + 32 * j);
-    } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) raw[j] = make_uint4(0, 0, 0, 0);
-    }
-    // (while the row loads are in flight) the linear's split-K counters and sum buffer start at zero for the GEMM that follows
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + tid; i < n_zero16;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-        zero16[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (tid < rows) s_amax[tid] = 0u;
-    float2 a[4][4];
+// Layout A from the four loaded 16-byte chunks (8 fp16 each), then the
+// butterfly stages on index bits 1, 2, 5, 6.  With `stagger` set, register
+// chunk j holds the group's chunk j ^ 1 (a warp's staggered shared-memory
+// reads then hit distinct banks); the bit-5 stage puts the pair back in
+// natural order (x0 + x1 into chunk 0, x0 - x1 = -(x1 - x0) into chunk 1,
+// bit-identical to the unstaggered result).  Below b = 64 there is no bit-5
+// stage and the caller undoes the stagger in the transpose.
+template <int LOG2B>
+__device__ __forceinline__ void act_layout_a(const uint4 (&raw)[4], bool stagger, float2 (&a)[4][4]) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t ww[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
@@ -300,10 +270,15 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
         }
     }
     if (LOG2B > 5) {  // bit 5
+        const float2 sg = f2(stagger ? -1.0f : 1.0f);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            bfly2(a[0][k], a[1][k]);
-            bfly2(a[2][k], a[3][k]);
+#pragma unroll
+            for (int j = 0; j < 4; j += 2) {
+                const float2 s = __fadd2_rn(a[j][k], a[j + 1][k]);
+                a[j + 1][k] = __fmul2_rn(sub2(a[j][k], a[j + 1][k]), sg);
+                a[j][k] = s;
+            }
         }
     }
     if (LOG2B > 6) {  // bit 6
@@ -313,18 +288,25 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
             bfly2(a[1][k], a[3][k]);
         }
     }
-    // ---- A -> B: unit u = 2p + 8j + h holds elements 4u .. 4u + 3 = a[j][2h], a[j][2h+1]
+}
+
+// A -> B through the group's transpose buffer (jx: register chunk j is the
+// group's chunk j ^ jx), then the stages on bits 0, 3, 4 and (b = 256) bit 7.
+// Every lane of the warp must call it (bit 7 uses shuffles).
+template <int LOG2B>
+__device__ __forceinline__ void act_layout_b(const float2 (&a)[4][4], uint8_t *xbuf, int p, int jx, int lane,
+                                             float2 (&bv)[8][2]) {
+    // unit u = 2p + 8j + h holds elements 4u .. 4u + 3 = a[j][2h], a[j][2h+1]
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            *reinterpret_cast<float4 *>(xbuf + 16 * xpose_slot(2 * p + 8 * j + h)) =
+            *reinterpret_cast<float4 *>(xbuf + 16 * xpose_slot(2 * p + 8 * (j ^ jx) + h)) =
                 make_float4(a[j][2 * h].x, a[j][2 * h].y, a[j][2 * h + 1].x, a[j][2 * h + 1].y);
         }
     }
     __syncwarp();
-    // ---- layout B: b[m][c] = (x[32p + 4m + c], x[32p + 4m + c + 2])
-    float2 bv[8][2];
+    // layout B: b[m][c] = (x[32p + 4m + c], x[32p + 4m + c + 2])
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
         const float4 f = *reinterpret_cast<const float4 *>(xbuf + 16 * xpose_slot(8 * p + m));
@@ -363,37 +345,37 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
             }
         }
     }
-    // ---- row maximum of |y| (y = unnormalized rotation)
+}
+
+// max |y| over the thread's 32 values (y = unnormalized rotation).
+__device__ __forceinline__ float act_local_absmax(const float2 (&bv)[8][2]) {
     float amax = 0.0f;
 #pragma unroll
     for (int m = 0; m < 8; ++m)
 #pragma unroll
         for (int c = 0; c < 2; ++c) amax = absmax3(amax, bv[m][c].x, bv[m][c].y);
-    const int G = reduce_width(L);
-    for (int mm = 1; mm < G; mm <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, mm));
-    // max|x~| = fp32(max|y| * rsqrt(b)) (rounding is monotone), s = fp32(that / qmax);
-    // code = rne(x~ * fp32(1/s)) with x~ = y * rsqrt(b): one factor per row
+    return amax;
+}
+
+// The row's scale and code factor from its max |y|: max|x~| = fp32(max|y| *
+// rsqrt(b)) (rounding is monotone), s = fp32(that / qmax); the code of x~ =
+// y * rsqrt(b) is rne(x~ * fp32(1/s)), taken as rne(y * fac) with one factor
+// per row, fac = fp32(rsqrt(b) * fp32(1/s)).
+template <int LOG2B, int BITS>
+__device__ __forceinline__ float act_row_scale(float amax, float *fac) {
+    constexpr float qmax = BITS == 8 ? 127.0f : 7.0f;
     const float rb = rsqrt_block(LOG2B);
-    float fac1;
-    if (G == L) {
-        // the whole row lives in this warp: no block-wide step
-        if (!active) return;
-        const float sc = __fdiv_rn(__fmul_rn(amax, rb), qmax);
-        fac1 = sc == 0.0f ? 0.0f : __fmul_rn(rb, __frcp_rn(sc));
-        if (l == 0) x_scale[row] = sc;
-    } else {
-        __syncthreads();  // s_amax initialised
-        if (r < rows && (l & (G - 1)) == 0) atomicMax(&s_amax[r], __float_as_uint(amax));  // amax >= 0
-        __syncthreads();
-        if (active && l == 0) {
-            const float sc = __fdiv_rn(__fmul_rn(__uint_as_float(s_amax[r]), rb), qmax);
-            s_fac[r] = sc == 0.0f ? 0.0f : __fmul_rn(rb, __frcp_rn(sc));
-            x_scale[row] = sc;
-        }
-        __syncthreads();
-        if (!active) return;
-        fac1 = s_fac[r];
-    }
+    const float sc = __fdiv_rn(__fmul_rn(amax, rb), qmax);
+    *fac = sc == 0.0f ? 0.0f : __fmul_rn(rb, __frcp_rn(sc));
+    return sc;
+}
+
+// Quantizes the thread's 32 values (one fused multiply-add each onto the
+// integer grid, see quant_clamped) and stores them: 32 bytes at element
+// 128g + 32p of the row, or 16 bytes of packed int4.
+template <int BITS, bool PACKED>
+__device__ __forceinline__ void act_store_codes(float2 (&bv)[8][2], float fac1, void *Xq, int64_t row, int K, int g,
+                                                int p) {
     const float2 fac = f2(fac1);
 #pragma unroll
     for (int m = 0; m < 8; ++m)
@@ -422,6 +404,139 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
         }
         uint8_t *dst = static_cast<uint8_t *>(Xq) + row * (K / 2) + 64 * g + 16 * p;
         *reinterpret_cast<uint4 *>(dst) = make_uint4(nb[0], nb[1], nb[2], nb[3]);
+    }
+}
+
+// BITS fixes the code range (8: [-127, 127], 4: [-8, 7]); PACKED stores int4
+// codes two per byte, otherwise every code takes one byte.
+// One CTA handles `rows` consecutive rows with L = K/32 threads each (the
+// block is padded to a multiple of 32 threads; padding threads only join the
+// barriers).  Every thread issues its four 16-byte loads up front.
+template <int LOG2B, int BITS, bool PACKED>
+__global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__restrict__ X, int64_t M, int K,
+                                                                int rows, void *__restrict__ Xq,
+                                                                float *__restrict__ x_scale,
+                                                                uint4 *__restrict__ zero16,
+                                                                int64_t n_zero16) {
+    extern __shared__ __align__(16) uint8_t act_smem[];
+    __shared__ unsigned int s_amax[kMaxRowsPerCta];
+    __shared__ float s_fac[kMaxRowsPerCta];
+    const int L = K / kElemsPerThread;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int r = tid / L;
+    const int l = tid - r * L;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * rows + r;
+    const bool active = (r < rows) && (row < M);
+    const int g = l >> 2, p = l & 3;
+    uint8_t *xbuf = act_smem + (tid >> 2) * kXposeGroupBytes;
+
+    pdl_wait();  // X may come from, and Xq may still be read by, the previous kernel
+    pdl_launch_dependents();
+    uint4 raw[4];
+    if (active) {
+        const __half *src = X + row * K + 128 * g + 8 * p;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) raw[j] = ld_stream_v4(src + 32 * j);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) raw[j] = make_uint4(0, 0, 0, 0);
+    }
+    // (while the row loads are in flight) the linear's split-K counters and sum buffer start at zero for the GEMM that follows
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + tid; i < n_zero16;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        zero16[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (tid < rows) s_amax[tid] = 0u;
+    float2 a[4][4];
+    act_layout_a<LOG2B>(raw, false, a);
+    float2 bv[8][2];
+    act_layout_b<LOG2B>(a, xbuf, p, 0, lane, bv);
+    float amax = act_local_absmax(bv);
+    const int G = reduce_width(L);
+    for (int mm = 1; mm < G; mm <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, mm));
+    float fac1;
+    if (G == L) {
+        // the whole row lives in this warp: no block-wide step
+        if (!active) return;
+        const float sc = act_row_scale<LOG2B, BITS>(amax, &fac1);
+        if (l == 0) x_scale[row] = sc;
+    } else {
+        __syncthreads();  // s_amax initialised
+        if (r < rows && (l & (G - 1)) == 0) atomicMax(&s_amax[r], __float_as_uint(amax));  // amax >= 0
+        __syncthreads();
+        if (active && l == 0) {
+            float f;
+            x_scale[row] = act_row_scale<LOG2B, BITS>(__uint_as_float(s_amax[r]), &f);
+            s_fac[r] = f;
+        }
+        __syncthreads();
+        if (!active) return;
+        fac1 = s_fac[r];
+    }
+    act_store_codes<BITS, PACKED>(bv, fac1, Xq, row, K, g, p);
+}
+
+// ---- the fused linear's activation warps ------------------------------------
+//
+// The same rotation in the register layout of fwht_block (thread l of the
+// row: element 128g + 8p + 32j + e, v[h][e] = (chunk h, chunk h + 2)), with no
+// shared memory: index bits 3 and 4 go between lanes l^1 and l^2.  The stages
+// run in the order of the activation kernel above (bits 1, 2, 5, 6, 0, 3, 4,
+// 7), so every sum is rounded in the same sequence and the codes are
+// bit-identical to that kernel's.
+template <int LOG2B>
+__device__ __forceinline__ void fwht_act_order(float2 (&v)[2][8], int lane) {
+#pragma unroll
+    for (int k = 1; k < 3; ++k) {  // bits 1, 2: e ^ m inside a chunk
+        if (k < LOG2B) {
+            const int m = 1 << k;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (!(e & m)) bfly2(v[h][e], v[h][e | m]);
+        }
+    }
+    if (LOG2B > 5) {  // bit 5: chunk pairs (0,1) and (2,3) -> h = 0 vs h = 1
+#pragma unroll
+        for (int e = 0; e < 8; ++e) bfly2(v[0][e], v[1][e]);
+    }
+    if (LOG2B > 6) {  // bit 6: chunk j vs j + 2 -> inside each float2
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float a = v[h][e].x, b = v[h][e].y;
+                v[h][e] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+            }
+    }
+    if (LOG2B > 0) {  // bit 0
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) bfly2(v[h][e], v[h][e + 1]);
+    }
+    if (LOG2B > 3) lane_stage(v, lane, 1);
+    if (LOG2B > 4) lane_stage(v, lane, 2);
+    if (LOG2B > 7) lane_stage(v, lane, 4);
+}
+
+// The thread's 32 fp16 elements (four 16-byte chunks j, 8 each) in fwht_block's layout.
+__device__ __forceinline__ void raw_to_v(const uint4 (&raw)[4], float2 (&v)[2][8]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t ww[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ww[k]));
+            if (j < 2) {
+                v[j][2 * k].x = f.x;
+                v[j][2 * k + 1].x = f.y;
+            } else {
+                v[j - 2][2 * k].y = f.x;
+                v[j - 2][2 * k + 1].y = f.y;
+            }
+        }
     }
 }
 

@@ -351,6 +351,11 @@ def test_linear_split_k_bit_exact(M, N, K, bits):
     ws_big = torch.empty(big, dtype=torch.uint8, device="cuda")
     y_ref = host(fn(Xd, Wq, sw, 128, bias=bd, workspace=ws_small))
     outs = [host(fn(Xd, Wq, sw, 128, bias=bd, workspace=ws_big)) for _ in range(3)]
+    # the two-launch form on the large workspace takes the split plans even where
+    # the linear runs fused
+    for _ in range(2):
+        cr.convrot_linear_quant_act(Xd, 128, bits, ws_big)
+        outs.append(host(cr.convrot_linear_gemm(ws_big, M, K, bits, Wq, sw, bias=bd)))
     for y in outs:
         assert np.array_equal(y.view(np.uint16), y_ref.view(np.uint16))
     # the workspace starts with the activation codes (one per byte) and, at the

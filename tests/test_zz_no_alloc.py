@@ -42,6 +42,29 @@ def test_noalloc_linear_matches_workspace_linear_two_calls_in_a_row():
         assert np.array_equal(y.cpu().numpy().view(np.uint16), y_ref.cpu().numpy().view(np.uint16))
 
 
+@pytest.mark.parametrize("M", [16, 1])
+def test_noalloc_linear_few_tokens_two_calls_in_a_row(M):
+    """Few tokens: 16 tokens take the feature-major GEMM with its K loop split
+    across SMs, whose counters and int32 sum buffer then live in the built-in
+    array too; one token takes the weight-streaming GEMM.  Two calls in a row
+    (the split state must be zero again for the second) equal the workspace
+    linear bit for bit."""
+    K = N = 4096
+    X = torch.from_numpy(wl.activations(M, K, 0.01, 30.0, seed=M)).cuda()
+    W = torch.from_numpy(wl.weight(N, K, 0.01, seed=M + 1)).cuda()
+    Wq, sw = cr.convrot_quantize_weight(W, 128, 8, cr.CLIP_MSE)
+    plan = cr.convrot_linear_plan(M, K, N, 8, 128, 16 << 20)
+    if M == 16:
+        assert plan["gemm_kind"] == 1 and plan["k_splits"] > 1, plan
+    else:
+        assert plan["gemm_kind"] == 2, plan
+    y_ref = cr.convrot_linear_w8a8(X, Wq, sw, 128)
+    for _ in range(2):
+        y = cr.convrot_linear_w8a8_noalloc(X, Wq, sw, 128)
+        cr.convrot_device_status()
+        assert np.array_equal(y.cpu().numpy().view(np.uint16), y_ref.cpu().numpy().view(np.uint16))
+
+
 def test_noalloc_linear_refuses_more_than_its_array():
     lib = cr.load_library()
     M, K, N = 16384, 4096, 64  # 64 MiB of codes: beyond the 16 MiB array
