@@ -72,7 +72,8 @@ def load_peaks():
 # ------------------------------------------------------------------------------------------ traffic
 
 CSRC = os.path.join(ROOT, "rotated_bit_quantized_block_b200", "csrc")
-GEMM_SOURCES = ("gemm_tcgen05.cuh", "device_utils.cuh")
+# (the GEMM kernels with activation warps, and the fused small-M kernel, run the rotation code too)
+GEMM_SOURCES = ("gemm_tcgen05.cuh", "gemv.cuh", "rotate_quant.cuh", "device_utils.cuh")
 ACT_SOURCES = ("rotate_quant.cuh", "device_utils.cuh")
 
 
@@ -448,45 +449,52 @@ def measure_workload(w, reps, stream, steps, peaks, clock_index=None, warmup=3):
         calls = [(lambda st, it=it: linear_call(w, it, st)) for it in items] * 2
         act = [(lambda st, it=it: cr.convrot_linear_quant_act(it["X"], w.block, bits, it["ws"], stream=st))
                for it in items] * 2
-        gemm = [(lambda st, it=it: cr.convrot_linear_gemm(it["ws"], w.M, lin.K, bits, it["Wq"], it["sw"], None,
-                                                          it["Y"], stream=st)) for it in items] * 2
+        if plan["weights_widened"]:
+            # the W4A4 linear's GEMM multiplies the weights its activation launch widened
+            # to int8 codes; they follow the int8-weight plan's part of the workspace
+            off = cr.convrot_linear_workspace_bytes(w.M, lin.K, lin.N, 8)
+            for it in items:
+                cr.convrot_linear_w4a4(it["X"], it["Wq"], it["sw"], w.block, None, it["Y"], it["ws"], stream)
+            gw = [it["ws"][off: off + lin.N * lin.K].view(torch.int8).view(lin.N, lin.K) for it in items]
+            gemm = [(lambda st, it=it, g=g: cr.convrot_linear_gemm(it["ws"], w.M, lin.K, 8, g, it["sw"], None,
+                                                                   it["Y"], stream=st))
+                    for it, g in zip(items, gw)] * 2
+        else:
+            gemm = [(lambda st, it=it: cr.convrot_linear_gemm(it["ws"], w.M, lin.K, bits, it["Wq"], it["sw"], None,
+                                                              it["Y"], stream=st)) for it in items] * 2
         t_lin, t_act, t_gemm = graph_ms(calls, stream), graph_ms(act, stream), graph_ms(gemm, stream)
         per[lin.name] = {"plan": plan, "linear_ms": t_lin, "act_ms": t_act, "gemm_ms": t_gemm}
+        if plan["fused_available"]:
+            # the rotation fused into the GEMM kernel (convrot_linear_w8a8_fused), for comparison
+            fused = [(lambda st, it=it: cr.convrot_linear_w8a8_fused(it["X"], it["Wq"], it["sw"], w.block, None,
+                                                                     it["Y"], it["ws"], st)) for it in items] * 2
+            per[lin.name]["fused_ms"] = graph_ms(fused, stream)
     cr.convrot_device_status(stream)
 
     ops = w.ops()
     lin_ms = sum(v["linear_ms"] for v in per.values())
-    # the dominant kernel: the fused linear kernel where a linear is one launch,
-    # otherwise its GEMM (the activation launch is reported under rotate_quant)
-    dom_ms = sum(v["linear_ms"] if v["plan"]["fused"] else v["gemm_ms"] for v in per.values())
+    # the dominant kernel: the GEMM (the activation launch is reported under rotate_quant)
+    dom_ms = sum(v["gemm_ms"] for v in per.values())
     int8_peak = 2.0 * peaks["bf16_tflops"]  # dense int8 = 2 x dense bf16 (4.5 vs 2.25 POPS nominal)
     if all(v["plan"]["gemm_kind"] == 2 for v in per.values()):
-        # the fewest tokens: bound by reading the weights; the fused kernel also
-        # reads X, the unfused one the activation codes
-        moved = sum(linear_bytes(w, l) - (0 if per[l.name]["plan"]["fused"] else w.M * l.K) for l in w.linears)
+        # the fewest tokens: bound by reading the weights (and the activation codes)
+        moved = sum(linear_bytes(w, l) - w.M * l.K for l in w.linears)
         achieved = moved / (dom_ms / 1e3) / 1e9
-        fused = all(v["plan"]["fused"] for v in per.values())
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"],
-                "kernel": ("gemv_fused (rotate+quant in every CTA, weight-streaming dp4a)" if fused
-                           else "gemv_i8 (weight-streaming, dp4a)"),
+                "frac": achieved / peaks["hbm_gbs"], "kernel": "gemv_i8 (weight-streaming, dp4a)",
                 "peak_note": f"{peaks['source']} HBM copy bandwidth"}
     else:
         achieved = ops / (dom_ms / 1e3) / 1e12
-        fused = all(v["plan"]["fused"] for v in per.values())
         roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
                 "frac": achieved / int8_peak,
-                "kernel": ("gemm_i8_tcgen05 with the fused rotate+quant prologue (int8 x int8 -> int32 in TMEM, "
-                           "dequant epilogue)" if fused else "gemm_i8_tcgen05 (int8 x int8 -> int32, dequant epilogue)"),
+                "kernel": "gemm_i8_tcgen05 (int8 x int8 -> int32 in TMEM, dequant epilogue)",
                 "peak_note": f"dense int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s"}
     roof.update({
         "timing": "each linear alone: CUDA graph of back-to-back launches over the rotating buffer sets, "
                   "CUDA events on the launching stream around the replay",
-        "per_linear_us": {n: round(1e3 * (v["linear_ms"] if v["plan"]["fused"] else v["gemm_ms"]), 2)
-                          for n, v in per.items()},
-        "per_linear_frac": {l.name: round(2 * w.M * l.K * l.N / ((per[l.name]["linear_ms"] if per[l.name]["plan"]["fused"]
-                                                                   else per[l.name]["gemm_ms"]) / 1e3) / 1e12
-                                          / int8_peak, 3) for l in w.linears},
+        "per_linear_us": {n: round(1e3 * v["gemm_ms"], 2) for n, v in per.items()},
+        "per_linear_frac": {l.name: round(2 * w.M * l.K * l.N / (per[l.name]["gemm_ms"] / 1e3) / 1e12 / int8_peak, 3)
+                            for l in w.linears},
     })
     act_total_ms = sum(v["act_ms"] for v in per.values())
     act_gbs = sum(act_bytes(w, l) for l in w.linears) / (act_total_ms / 1e3) / 1e9
@@ -498,12 +506,15 @@ def measure_workload(w, reps, stream, steps, peaks, clock_index=None, warmup=3):
           "per_linear_us": {n: round(1e3 * v["act_ms"], 2) for n, v in per.items()},
           "per_linear_gbs": {l.name: round(act_bytes(w, l) / (per[l.name]["act_ms"] / 1e3) / 1e9, 1)
                              for l in w.linears}}
+    fused_cmp = {n: {"fused_us": round(1e3 * v["fused_ms"], 2), "two_launch_us": round(1e3 * v["linear_ms"], 2)}
+                 for n, v in per.items() if "fused_ms" in v}
     return {
+        "fused_linear": fused_cmp,
         "elapsed_ms": elapsed_ms, "ms_per_step": elapsed_ms / steps, "clocks": clocks,
         "tokens_per_s": w.M * steps / (elapsed_ms / 1e3), "tops": ops * steps / (elapsed_ms / 1e3) / 1e12,
         "roofline": roof, "rotate_quant": rq,
         "kernel_us_per_step": round(1e3 * lin_ms, 2),
-        "two_launch_us_per_step": round(1e3 * sum(v["act_ms"] + v["gemm_ms"] for v in per.values()), 2),
+        "act_plus_gemm_us_per_step": round(1e3 * sum(v["act_ms"] + v["gemm_ms"] for v in per.values()), 2),
         "launches_per_step": sum(v["plan"]["launches"] for v in per.values()),
         "plans": {n: v["plan"] for n, v in per.items()},
     }
@@ -637,7 +648,8 @@ def ours_arm(args, w, rank, world, local_rank):
         "roofline": roofline,
         "rotate_quant": rotate_quant,
         "kernel_us_per_step": m["kernel_us_per_step"],
-        "two_launch_us_per_step": m["two_launch_us_per_step"],
+        "act_plus_gemm_us_per_step": m["act_plus_gemm_us_per_step"],
+        "fused_linear": m["fused_linear"],
         "plans": m["plans"],
         "offline_weight_quant_ms": weight_quant_ms,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -658,12 +670,14 @@ def ours_arm(args, w, rank, world, local_rank):
             sm = measure_workload(sw_, sreps, stream, args.sub_steps, peaks)
             subs[name] = {
                 "tokens_per_s": sm["tokens_per_s"], "tops": sm["tops"], "us_per_step": 1e3 * sm["ms_per_step"],
-                "kernel_us_per_step": sm["kernel_us_per_step"], "two_launch_us_per_step": sm["two_launch_us_per_step"],
+                "kernel_us_per_step": sm["kernel_us_per_step"],
+                "act_plus_gemm_us_per_step": sm["act_plus_gemm_us_per_step"], "fused_linear": sm["fused_linear"],
                 "roofline_bound": sm["roofline"]["bound"], "roofline_frac": sm["roofline"]["frac"],
                 "roofline_achieved": sm["roofline"]["achieved"], "roofline_unit": sm["roofline"]["unit"],
                 "per_linear_frac": sm["roofline"]["per_linear_frac"],
                 "rotate_quant_frac": sm["rotate_quant"]["frac"], "rotate_quant_gbs": sm["rotate_quant"]["achieved"],
-                "plans": {n: f"{'fused ' if p['fused'] else ''}{['token-major', 'feature-major', 'gemv'][p['gemm_kind']]}"
+                "plans": {n: f"{'widened int4 weights, ' if p['weights_widened'] else ''}"
+                             f"{['token-major', 'feature-major', 'gemv'][p['gemm_kind']]}"
                              f"{' bn' + str(p['tile_n']) if p['tile_n'] else ''}{' pair' if p['cta_pair'] else ''}"
                              f"{' stream-K' if p['stream_k'] else ''}{' split' + str(p['k_splits']) if p['k_splits'] > 1 else ''}"
                           for n, p in sm["plans"].items()},

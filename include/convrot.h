@@ -145,7 +145,9 @@ size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
  * (128 x 256) that the first of them stores in a slot of this workspace.
  * Size: convrot_workspace_bytes(M, K, bits) plus 2 KB of split-K counters plus
  * that buffer (rounded up to 256 bytes) or (SMs + 1) partial-tile slots of
- * 128 KB.  The activation half of the linear zeroes the counters and the M x N
+ * 128 KB.  For W4A4 over more than 128 tokens it also holds the weights
+ * widened to int8 codes (N*K bytes, after the split buffer of the int8-weight
+ * plan): see convrot_linear_w4a4.  The activation half of the linear zeroes the counters and the M x N
  * buffer; the GEMM half leaves both zeroed again (the partial-tile slots are
  * written before they are read and need no zeroing).  With only the minimum
  * workspace the linears never split.  Depends on the current device's SM
@@ -175,7 +177,11 @@ convrot_status_t convrot_linear_w8a8(const void *X, int64_t M, int64_t K, const 
  * uses W4A4 operations"; INT8 multiplication on hardware without INT4 MMA).
  * As convrot_linear_w8a8 with Wq the packed int4 codes [N x K/2] from
  * convrot_quantize_weight(bits = 4) and workspace >=
- * convrot_workspace_bytes(M, K, 4).
+ * convrot_workspace_bytes(M, K, 4).  With more than 128 tokens and a workspace
+ * of convrot_linear_workspace_bytes(M, K, N, 4), the activation launch also
+ * widens the packed weights once to int8 codes in the workspace and the GEMM
+ * multiplies those (the same integers, so the same output); otherwise the GEMM
+ * widens the packed tiles in shared memory.
  */
 convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const uint8_t *Wq,
                                      const float *w_scale, int64_t N, const void *bias, int block, void *Y,
@@ -184,36 +190,53 @@ convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const 
 /*
  * How convrot_linear_w8a8 / convrot_linear_w4a4 would run a call of these
  * sizes with a workspace of workspace_bytes on the current device (no launch):
- *   fused      1: the linear rotates and quantizes inside its GEMM kernel.
- *              For the fewest tokens (the weight-streaming plan, block 128, K
- *              a multiple of 512 up to 8192) every CTA rotates the few token
- *              rows itself into shared memory while its first weights load.
- *              For more than 128 tokens (W8A8, block 128, K <= 2048, workspace
- *              >= convrot_linear_workspace_bytes) activation warps in the
- *              GEMM's CTAs rotate and quantize the tokens into the workspace
- *              beside the tensor-core main loop, which loads each 128-token
- *              panel once all of its rows are done; a tiny kernel zeroing the
- *              panel counters goes first.  0: the activation kernel, then the
- *              GEMM.
- *   launches   kernels per call.
+ *   launches   kernels per call (the activation kernel, then the GEMM).
  *   gemm_kind  0: token-major tensor-core tiles (128 tokens x tile_n
  *              features); 1: feature-major tiles (128 features x tile_n
  *              tokens); 2: the weight-streaming kernel (dp4a).
  *   cta_pair / stream_k / k_splits: CTA pairs (cta_group::2), stream-K shares,
  *              K slices of the feature-major split.
- * (Civarchive ConvRot release, "Future improvements": fusion of the steps.)
+ *   fused_available  1 if convrot_linear_w8a8_fused accepts the call (W8A8).
+ *   weights_widened  1 if the W4A4 linear widens its weights to int8 codes in
+ *              the workspace and runs the int8-weight GEMM (the fields above
+ *              then describe that GEMM).
  */
 typedef struct {
     int launches;
-    int fused;
     int gemm_kind;
     int tile_n;
     int cta_pair;
     int stream_k;
     int k_splits;
+    int fused_available;
+    int weights_widened;
 } convrot_linear_plan_t;
 convrot_status_t convrot_linear_plan(int64_t M, int64_t K, int64_t N, int bits, int block, size_t workspace_bytes,
                                      convrot_linear_plan_t *plan);
+
+/*
+ * W8A8 ConvRot linear with the rotation fused into the GEMM kernel
+ * (civarchive ConvRot release, "Future improvements": fusion of the steps).
+ * Same arguments and results as convrot_linear_w8a8 -- the codes, scales and
+ * Y are bit-identical -- but the GEMM's CTAs carry eight activation warps that
+ * rotate and quantize units of tokens into the workspace beside the
+ * tensor-core main loop; the producer loads a 128-token panel's codes once
+ * every unit touching it has been counted into the panel's counter.  A tiny
+ * kernel zeroing the counters precedes it.  On B200 the two-launch linear
+ * measured faster at every shape tried (the activation kernel then has the
+ * whole GPU), so convrot_linear_w8a8 does not use this path.
+ *   Supported: more than 128 tokens, block 128, K <= 2048, at most 512
+ *   panels of 128 tokens; otherwise CONVROT_ERR_UNSUPPORTED.
+ *   workspace  at least convrot_workspace_bytes(M, K, 8) + 2048 bytes (the
+ *              panel counters follow the scales);
+ *              convrot_linear_workspace_bytes(M, K, N, 8) always suffices.
+ * The CTAs wait for one another (bounded): every CTA must be co-resident, which
+ * the grid (at most one CTA or CTA pair per SM) ensures when no other kernel
+ * holds SMs for the whole run of this one.
+ */
+convrot_status_t convrot_linear_w8a8_fused(const void *X, int64_t M, int64_t K, const int8_t *Wq,
+                                           const float *w_scale, int64_t N, const void *bias, int block, void *Y,
+                                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * The two launches of convrot_linear_w8a8 / convrot_linear_w4a4, callable

@@ -25,15 +25,15 @@ EXPORTED = (
     "convrot_device_status", "convrot_status_string", "convrot_last_error", "convrot_version",
     "convrot_linear_w8a8_noalloc", "convrot_linear_quant_act", "convrot_linear_gemm",
     "convrot_linear_workspace_bytes", "convrot_tensorwise_workspace_bytes", "convrot_quantize_weight_tensorwise",
-    "convrot_test_abandoned_wait", "convrot_linear_plan",
+    "convrot_test_abandoned_wait", "convrot_linear_plan", "convrot_linear_w8a8_fused",
 )
 
 
 class LinearPlan(ctypes.Structure):
     """convrot_linear_plan_t: how a linear call runs (see include/convrot.h)."""
-    _fields_ = [("launches", ctypes.c_int), ("fused", ctypes.c_int), ("gemm_kind", ctypes.c_int),
-                ("tile_n", ctypes.c_int), ("cta_pair", ctypes.c_int), ("stream_k", ctypes.c_int),
-                ("k_splits", ctypes.c_int)]
+    _fields_ = [("launches", ctypes.c_int), ("gemm_kind", ctypes.c_int), ("tile_n", ctypes.c_int),
+                ("cta_pair", ctypes.c_int), ("stream_k", ctypes.c_int), ("k_splits", ctypes.c_int),
+                ("fused_available", ctypes.c_int), ("weights_widened", ctypes.c_int)]
 
     def as_dict(self):
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -68,6 +68,7 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
             "convrot_quantize_weight_tensorwise": (i32, [P, i32, i64, i64, i32, i32, i32, P, P, P, sz, P]),
             "convrot_linear_w8a8": (i32, [P, i64, i64, P, P, i64, P, i32, P, P, sz, P]),
             "convrot_linear_w4a4": (i32, [P, i64, i64, P, P, i64, P, i32, P, P, sz, P]),
+            "convrot_linear_w8a8_fused": (i32, [P, i64, i64, P, P, i64, P, i32, P, P, sz, P]),
             "convrot_gemm_w8a8": (i32, [P, P, i64, P, P, i64, i64, P, P, P, P]),
             "convrot_gemm_w4a4": (i32, [P, P, i64, P, P, i64, i64, P, P, P, P]),
             "convrot_linear_w8a8_noalloc": (i32, [P, i64, i64, P, P, i64, P, i32, P, P]),
@@ -208,6 +209,11 @@ def _linear(fn_name, bits, X, Wq, w_scale, block, bias, Y, workspace, stream):
 def convrot_linear_w8a8(X, Wq, w_scale, block, bias=None, Y=None, workspace=None, stream=None):
     """Y = ConvRot W8A8 linear of X (fp16) with int8 weight codes Wq (N x K)."""
     return _linear("convrot_linear_w8a8", 8, X, Wq, w_scale, block, bias, Y, workspace, stream)
+
+
+def convrot_linear_w8a8_fused(X, Wq, w_scale, block, bias=None, Y=None, workspace=None, stream=None):
+    """The W8A8 linear as one GEMM kernel whose activation warps rotate and quantize X."""
+    return _linear("convrot_linear_w8a8_fused", 8, X, Wq, w_scale, block, bias, Y, workspace, stream)
 
 
 def convrot_linear_w4a4(X, Wq, w_scale, block, bias=None, Y=None, workspace=None, stream=None):

@@ -225,9 +225,19 @@ cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Extra grid-stride work of the activation launch: zeroing split-K state, and
+// widening the W4A4 linear's packed weights to int8 codes.
+struct ActExtras {
+    uint4 *zero16 = nullptr;
+    int64_t n_zero16 = 0;
+    const uint4 *w_packed = nullptr;
+    uint4 *w_wide = nullptr;
+    int64_t n_w16 = 0;
+};
+
 template <int LOG2B, int BITS, bool PACKED>
 void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms, int dev,
-                uint4 *zero16, int64_t n_zero16) {
+                const ActExtras &ex) {
     auto kern = convrot::act_rotate_quant_kernel<LOG2B, BITS, PACKED>;
     {
         static bool configured[kMaxDevices];
@@ -244,22 +254,23 @@ void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaSt
     act_geometry(kern, sms, M, K, &R, &T);
     const int64_t grid = (M + R - 1) / R;
     launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(T), static_cast<size_t>(convrot::act_smem_bytes(T)), st,
-               static_cast<const __half *>(X), M, static_cast<int>(K), R, Xq, xs, zero16, n_zero16);
+               static_cast<const __half *>(X), M, static_cast<int>(K), R, Xq, xs, ex.zero16, ex.n_zero16, ex.w_packed,
+               ex.w_wide, ex.n_w16);
 }
 
 template <int BITS, bool PACKED>
 void dispatch_act(int log2b, const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaStream_t st, int sms,
-                  int dev, uint4 *zw, int64_t nzw) {
+                  int dev, const ActExtras &ex) {
     switch (log2b) {
-        case 0: launch_act<0, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
-        case 1: launch_act<1, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
-        case 2: launch_act<2, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
-        case 3: launch_act<3, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
-        case 4: launch_act<4, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
-        case 5: launch_act<5, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
-        case 6: launch_act<6, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
-        case 7: launch_act<7, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
-        default: launch_act<8, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, zw, nzw); break;
+        case 0: launch_act<0, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, ex); break;
+        case 1: launch_act<1, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, ex); break;
+        case 2: launch_act<2, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, ex); break;
+        case 3: launch_act<3, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, ex); break;
+        case 4: launch_act<4, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, ex); break;
+        case 5: launch_act<5, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, ex); break;
+        case 6: launch_act<6, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, ex); break;
+        case 7: launch_act<7, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, ex); break;
+        default: launch_act<8, BITS, PACKED>(X, M, K, Xq, xs, st, sms, dev, ex); break;
     }
 }
 
@@ -300,11 +311,11 @@ void dispatch_weight(int log2b, const void *W, int dtype, int64_t N, int64_t K, 
 // packed: int4 codes two per byte (bits = 4 only); otherwise one byte per code.
 convrot_status_t rotate_quant_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, bool packed,
                                        void *Xq, float *x_scale, cudaStream_t st, int sms, int dev,
-                                       uint4 *zero16 = nullptr, int64_t n_zero16 = 0) {
+                                       const ActExtras &ex = ActExtras()) {
     const int log2b = ilog2(block);
-    if (bits == 8) dispatch_act<8, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev, zero16, n_zero16);
-    else if (packed) dispatch_act<4, true>(log2b, X, M, K, Xq, x_scale, st, sms, dev, zero16, n_zero16);
-    else dispatch_act<4, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev, zero16, n_zero16);
+    if (bits == 8) dispatch_act<8, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev, ex);
+    else if (packed) dispatch_act<4, true>(log2b, X, M, K, Xq, x_scale, st, sms, dev, ex);
+    else dispatch_act<4, false>(log2b, X, M, K, Xq, x_scale, st, sms, dev, ex);
     return launch_status("act_rotate_quant");
 }
 
@@ -422,6 +433,20 @@ struct FusePrologue {
 
 // Block sizes the fused linear is built for (others take two launches).
 constexpr bool fuse_block_supported(int log2b) { return log2b == 7; }
+
+// The W4A4 linear over more than 128 tokens (token-major tiles) widens its
+// packed weights once per call to int8 codes in the workspace, in its
+// activation launch, and runs the int8-weight GEMM on them: every M tile would
+// otherwise widen the same weight tiles again in shared memory.  The products
+// are the same integers either way.
+bool w4_prewidens(int64_t M) { return M > kSwapMaxTokens; }
+
+// Offset of the widened weights: after the codes, scales, counters and the
+// split buffer of the int8-weight plan.
+size_t w4_wide_offset(int sms, int64_t M, int64_t K, int64_t N) {
+    return round256(static_cast<size_t>(M) * K) + round256(static_cast<size_t>(M) * 4) + kCounterBytes +
+           split_buffer_bytes(plan_gemm(sms, M, N, K, true, false), M, N);
+}
 
 // Xc: activation codes (M x K), Wc: weight codes (N x K); A4 / B4 of Cfg refer
 // to the MMA's operands (token-major: A = activations; feature-major: A = weights).
@@ -607,52 +632,6 @@ convrot_status_t check_gemm_args(const void *Xq, const float *xs, int64_t M, con
     return ok();
 }
 
-// The fused small-M linear (rotate + quantize in every CTA, then the weight
-// stream): for the plans that take the weight-streaming GEMM, block 128 and
-// K a multiple of 512 up to 8192.
-static bool fused_gemv_plan(int sms, int64_t M, int64_t K, int64_t N, int bits, int block, GemmPlan *plan) {
-    if (!fuse_block_supported(ilog2(block)) || K % convrot::kGemvChunk != 0 || K > convrot::kGemvFusedMaxK) return false;
-    const GemmPlan p = plan_gemm(sms, M, N, K, false, bits == 4);
-    if (!p.gemv) return false;
-    *plan = p;
-    return true;
-}
-
-template <bool W4, int MT>
-convrot_status_t launch_gemv_fused_mt(int dev, int sms, const void *X, const void *Wc, int64_t M, int64_t N,
-                                      int64_t K, const float *sw, const void *bias, void *Y, int8_t *xq,
-                                      float *xs, cudaStream_t st) {
-    auto kern = convrot::gemv_fused_kernel<W4, MT, 7>;
-    {
-        static std::mutex mu;
-        static bool done[kMaxDevices] = {};
-        std::lock_guard<std::mutex> lock(mu);
-        if (!done[dev]) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 convrot::gemv_fused_smem_bytes(MT, convrot::kGemvFusedMaxK));
-            CR_REQUIRE(e == cudaSuccess, CONVROT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-            done[dev] = true;
-        }
-    }
-    const int64_t groups = (N + 3) / 4;
-    const int grid = static_cast<int>(groups < sms ? groups : sms);
-    launch_pdl(kern, dim3(grid), dim3(convrot::kGemvFusedThreads),
-               static_cast<size_t>(convrot::gemv_fused_smem_bytes(MT, static_cast<int>(K))), st,
-               static_cast<const __half *>(X), static_cast<const uint8_t *>(Wc), sw, static_cast<const __half *>(bias),
-               static_cast<__half *>(Y), xq, xs, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
-    return launch_status("gemv_fused");
-}
-
-template <bool W4>
-convrot_status_t launch_gemv_fused(int dev, int sms, const void *X, const void *Wc, int64_t M, int64_t N, int64_t K,
-                                   const float *sw, const void *bias, void *Y, int8_t *xq, float *xs,
-                                   cudaStream_t st) {
-    if (M <= 1) return launch_gemv_fused_mt<W4, 1>(dev, sms, X, Wc, M, N, K, sw, bias, Y, xq, xs, st);
-    if (M <= 2) return launch_gemv_fused_mt<W4, 2>(dev, sms, X, Wc, M, N, K, sw, bias, Y, xq, xs, st);
-    if (M <= 4) return launch_gemv_fused_mt<W4, 4>(dev, sms, X, Wc, M, N, K, sw, bias, Y, xq, xs, st);
-    return launch_gemv_fused_mt<W4, 8>(dev, sms, X, Wc, M, N, K, sw, bias, Y, xq, xs, st);
-}
-
 }  // namespace
 
 // =============================================================================
@@ -697,6 +676,7 @@ size_t convrot_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits)
         cudaGetLastError();
     }
     if (M == 0 || N == 0 || K % 128 != 0 || K < 128) return base + kCounterBytes;
+    if (bits == 4 && w4_prewidens(M)) return w4_wide_offset(sms, M, K, N) + round256(static_cast<size_t>(N) * K);
     return base + kCounterBytes + split_buffer_bytes(plan_gemm(sms, M, N, K, true, bits == 4), M, N);
 }
 
@@ -824,8 +804,11 @@ static convrot_status_t check_workspace(const void *workspace, size_t workspace_
 // n_features >= 0: the GEMM half's N is known, so exactly the split-K state it
 // will use is zeroed; otherwise everything after the codes and scales, up to
 // the largest split buffer a GEMM over M tokens can use.
+// wide: the packed int4 weights (N x K/2) to widen into the workspace (see
+// w4_prewidens), or null.
 static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, void *workspace,
-                                        size_t workspace_bytes, cudaStream_t st, int64_t n_features = -1) {
+                                        size_t workspace_bytes, cudaStream_t st, int64_t n_features = -1,
+                                        const void *wide = nullptr) {
     CR_REQUIRE(X != nullptr, CONVROT_ERR_INVALID_ARG, "null pointer argument");
     CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
     CR_TRY(check_workspace(workspace, workspace_bytes, M, K, bits));
@@ -844,16 +827,23 @@ static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int
         size_t cap;
         if (n_features >= 0) {
             // (stream-K partial slots are written before they are read: only the counters)
-            const GemmPlan p = plan_gemm(info->sms, M, n_features, K, true, bits == 4);
+            const GemmPlan p = plan_gemm(info->sms, M, n_features, K, true, bits == 4 && wide == nullptr);
             cap = kCounterBytes + (p.streamk > 0 ? 0 : split_buffer_bytes(p, M, n_features));
         } else {
             cap = kCounterBytes + (M <= kSwapMaxTokens ? round256(static_cast<size_t>(M) * kMaxSplitFeatures * 4) : 0);
         }
         zero_bytes = (workspace_bytes - base < cap ? workspace_bytes - base : cap) & ~size_t(15);
     }
-    return rotate_quant_act_impl(X, M, K, block, bits, false, xq, xs, st, info->sms, dev,
-                                 zero_bytes ? reinterpret_cast<uint4 *>(counters) : nullptr,
-                                 static_cast<int64_t>(zero_bytes / 16));
+    ActExtras ex;
+    ex.zero16 = zero_bytes ? reinterpret_cast<uint4 *>(counters) : nullptr;
+    ex.n_zero16 = static_cast<int64_t>(zero_bytes / 16);
+    if (wide != nullptr) {
+        ex.w_packed = static_cast<const uint4 *>(wide);
+        ex.w_wide = reinterpret_cast<uint4 *>(static_cast<uint8_t *>(workspace) +
+                                              w4_wide_offset(info->sms, M, K, n_features));
+        ex.n_w16 = n_features * K / 32;  // 16 packed bytes (32 codes) per unit
+    }
+    return rotate_quant_act_impl(X, M, K, block, bits, false, xq, xs, st, info->sms, dev, ex);
 }
 
 // The GEMM plan of a linear's second launch: split K only when the workspace
@@ -903,50 +893,6 @@ static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace
                                     counters);
 }
 
-// One launch for the whole linear where the fused prologue applies (see
-// fused_plan).  *fused tells whether it ran.
-static convrot_status_t linear_fused_impl(int bits, const void *X, int64_t M, int64_t K, const void *Wq,
-                                          const float *w_scale, int64_t N, const void *bias, int block, void *Y,
-                                          void *workspace, size_t workspace_bytes, cudaStream_t st, bool *fused) {
-    *fused = false;
-    if (workspace == nullptr) return ok();
-    int dev;
-    DeviceInfo *info;
-    CR_TRY(current_device(&dev, &info));
-    GemmPlan p;
-    if (fused_gemv_plan(info->sms, M, K, N, bits, block, &p)) {
-        void *xq;
-        float *xs;
-        workspace_parts(workspace, M, K, &xq, &xs);
-        CR_TRY(check_gemm_args(xq, xs, M, Wq, w_scale, N, K, bias, Y));
-        *fused = true;
-        if (bits == 8)
-            return launch_gemv_fused<false>(dev, info->sms, X, Wq, M, N, K, w_scale, bias, Y,
-                                            static_cast<int8_t *>(xq), xs, st);
-        return launch_gemv_fused<true>(dev, info->sms, X, Wq, M, N, K, w_scale, bias, Y, static_cast<int8_t *>(xq),
-                                       xs, st);
-    }
-    if (!fused_plan(info->sms, M, K, N, bits, block, workspace_bytes, &p)) return ok();
-    const int log2b = ilog2(block);
-    CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
-    CR_REQUIRE(aligned(workspace, 16), CONVROT_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
-    void *xq;
-    float *xs;
-    unsigned int *counters;
-    workspace_parts(workspace, M, K, &xq, &xs, &counters);
-    CR_TRY(check_gemm_args(xq, xs, M, Wq, w_scale, N, K, bias, Y));
-    FusePrologue fz;
-    fz.X = X;
-    fz.log2b = log2b;
-    fz.panels = counters;
-    *fused = true;
-    // zero the panel counters (programmatic launch: overlaps the previous kernel's tail)
-    const int panels = static_cast<int>((M + 127) / 128);
-    launch_pdl(convrot::fuse_zero_kernel, dim3(1), dim3(256), 0, st, counters, panels);
-    CR_TRY(launch_status("fuse_zero"));
-    return launch_gemm_fused(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, st, p, fz);
-}
-
 static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t K, const void *Wq,
                                     const float *w_scale, int64_t N, const void *bias, int block, void *Y,
                                     void *workspace, size_t workspace_bytes, void *stream) {
@@ -954,12 +900,20 @@ static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t 
     CR_TRY(check_linear_shape(M, K, block, bits, N));
     if (M == 0 || N == 0) return ok();
     CR_REQUIRE(X && Wq && w_scale && Y, CONVROT_ERR_INVALID_ARG, "null pointer argument");
-    CR_TRY(check_workspace(workspace, workspace_bytes, M, K, bits));
-    CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    bool fused = false;
-    CR_TRY(linear_fused_impl(bits, X, M, K, Wq, w_scale, N, bias, block, Y, workspace, workspace_bytes, st, &fused));
-    if (fused) return ok();
+    if (bits == 4 && w4_prewidens(M) && workspace != nullptr) {
+        CR_REQUIRE(aligned(Wq, 16), CONVROT_ERR_ALIGNMENT, "Wq must be 16-byte aligned");
+        int dev;
+        DeviceInfo *info;
+        CR_TRY(current_device(&dev, &info));
+        const size_t off = w4_wide_offset(info->sms, M, K, N);
+        if (workspace_bytes >= off + round256(static_cast<size_t>(N) * K)) {
+            // the activation launch also widens the weights; the int8-weight GEMM follows
+            CR_TRY(linear_act_impl(X, M, K, block, 4, workspace, workspace_bytes, st, N, Wq));
+            const int8_t *wide = static_cast<const int8_t *>(workspace) + off;
+            return linear_gemm_impl(workspace, workspace_bytes, M, K, 8, wide, w_scale, N, bias, Y, st);
+        }
+    }
     CR_TRY(linear_act_impl(X, M, K, block, bits, workspace, workspace_bytes, st, N));
     return linear_gemm_impl(workspace, workspace_bytes, M, K, bits, Wq, w_scale, N, bias, Y, st);
 }
@@ -993,6 +947,49 @@ convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const 
                                      int64_t N, const void *bias, int block, void *Y, void *workspace,
                                      size_t workspace_bytes, void *stream) {
     return linear_impl(4, X, M, K, Wq, w_scale, N, bias, block, Y, workspace, workspace_bytes, stream);
+}
+
+convrot_status_t convrot_linear_w8a8_fused(const void *X, int64_t M, int64_t K, const int8_t *Wq,
+                                           const float *w_scale, int64_t N, const void *bias, int block, void *Y,
+                                           void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    CR_TRY(check_linear_shape(M, K, block, 8, N));
+    if (M == 0 || N == 0) return ok();
+    CR_REQUIRE(X && Wq && w_scale && Y, CONVROT_ERR_INVALID_ARG, "null pointer argument");
+    const size_t need = convrot_workspace_bytes(M, K, 8) + kCounterBytes;
+    CR_REQUIRE(workspace != nullptr && workspace_bytes >= need, CONVROT_ERR_WORKSPACE,
+               "workspace of %zu bytes given, %zu needed (codes, scales and the panel counters)", workspace_bytes,
+               need);
+    CR_REQUIRE(aligned(workspace, 16), CONVROT_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+    CR_REQUIRE(aligned(X, 16), CONVROT_ERR_ALIGNMENT, "X must be 16-byte aligned");
+    CR_REQUIRE(M > kSwapMaxTokens && block == 128 && K <= kFuseMaxK && (M + 127) / 128 <= convrot::kFuseMaxPanels,
+               CONVROT_ERR_UNSUPPORTED,
+               "the fused linear takes more than %lld tokens, block 128, K <= %lld and at most %d panels "
+               "(M = %lld, K = %lld, block = %d)",
+               static_cast<long long>(kSwapMaxTokens), static_cast<long long>(kFuseMaxK), convrot::kFuseMaxPanels,
+               static_cast<long long>(M), static_cast<long long>(K), block);
+    int dev;
+    DeviceInfo *info;
+    CR_TRY(current_device(&dev, &info));
+    GemmPlan p;
+    CR_REQUIRE(fused_plan(info->sms, M, K, N, 8, block, workspace_bytes, &p), CONVROT_ERR_UNSUPPORTED,
+               "no fused plan for M = %lld, N = %lld, K = %lld", static_cast<long long>(M), static_cast<long long>(N),
+               static_cast<long long>(K));
+    void *xq;
+    float *xs;
+    unsigned int *counters;
+    workspace_parts(workspace, M, K, &xq, &xs, &counters);
+    CR_TRY(check_gemm_args(xq, xs, M, Wq, w_scale, N, K, bias, Y));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // zero the panel counters (programmatic launch: overlaps the previous kernel's tail)
+    const int panels = static_cast<int>((M + 127) / 128);
+    launch_pdl(convrot::fuse_zero_kernel, dim3(1), dim3(256), 0, st, counters, panels);
+    CR_TRY(launch_status("fuse_zero"));
+    FusePrologue fz;
+    fz.X = X;
+    fz.log2b = ilog2(block);
+    fz.panels = counters;
+    return launch_gemm_fused(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, st, p, fz);
 }
 
 static convrot_status_t gemm_impl(bool w4, const void *Xq, const float *x_scale, int64_t M, const void *Wq,
@@ -1083,13 +1080,13 @@ convrot_status_t convrot_linear_plan(int64_t M, int64_t K, int64_t N, int bits, 
     int dev;
     DeviceInfo *info;
     CR_TRY(current_device(&dev, &info));
-    GemmPlan p;
-    const bool fused_gemv = fused_gemv_plan(info->sms, M, K, N, bits, block, &p);
-    const bool fused = fused_gemv || fused_plan(info->sms, M, K, N, bits, block, workspace_bytes, &p);
-    if (!fused) p = two_launch_plan(info->sms, M, N, K, bits, workspace_bytes);
-    // counter zeroing + fused GEMM, one fused weight-streaming kernel, or activation kernel + GEMM
-    plan->launches = fused_gemv ? 1 : 2;
-    plan->fused = fused ? 1 : 0;
+    const bool widened = bits == 4 && w4_prewidens(M) &&
+                         workspace_bytes >= w4_wide_offset(info->sms, M, K, N) + round256(static_cast<size_t>(N) * K);
+    const GemmPlan p = two_launch_plan(info->sms, M, N, K, widened ? 8 : bits, workspace_bytes);
+    GemmPlan pf;
+    plan->launches = 2;  // the activation kernel, then the GEMM
+    plan->weights_widened = widened ? 1 : 0;
+    plan->fused_available = (bits == 8 && fused_plan(info->sms, M, K, N, bits, block, workspace_bytes, &pf)) ? 1 : 0;
     plan->gemm_kind = p.gemv ? 2 : (p.swap ? 1 : 0);
     plan->tile_n = p.gemv ? 0 : p.bn;
     plan->cta_pair = p.pair ? 1 : 0;

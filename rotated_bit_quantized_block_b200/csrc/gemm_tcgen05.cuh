@@ -202,15 +202,15 @@ __global__ void __launch_bounds__(256) fuse_zero_kernel(unsigned int *counters, 
     pdl_launch_dependents();
 }
 
-// Rows per activation unit of `nt` threads (L = K/32 threads per row).
-__host__ __device__ __forceinline__ int fuse_unit_rows(int nt, int K) { return nt / (K / kElemsPerThread); }
-
-// Number of units that touch panel p (rows [128 p, min(128 p + 128, M))).
+// Number of units (RPR rows each) that touch panel p (rows [128 p, min(128 p + 128, M))).
 __device__ __forceinline__ uint32_t fuse_panel_units(int64_t M, int rpr, int64_t p) {
     const int64_t r0 = 128 * p;
     const int64_t r1 = (r0 + 128 < M ? r0 + 128 : M) - 1;
     return static_cast<uint32_t>(r1 / rpr - r0 / rpr + 1);
 }
+
+// Rows per activation unit of `nt` threads (L = K/32 threads per row).
+__host__ __device__ __forceinline__ int fuse_unit_rows(int nt, int K) { return nt / (K / kElemsPerThread); }
 
 // Waits (acquire, bounded) until panel p's counter shows all of its units.
 __device__ __forceinline__ bool fuse_panel_wait(const unsigned int *counters, int64_t M, int rpr, int64_t p,
@@ -237,6 +237,8 @@ __device__ __forceinline__ bool fuse_panel_wait(const unsigned int *counters, in
 // touches (release: the consumers acquire the counter, then fence the async
 // proxy before their TMA loads).  Rows spanning several warps meet in s_part
 // behind named barrier bar_id (all NT threads join it the same number of times).
+// (Counting per warp instead, with one release reduction per warp and panel and
+// no CTA-wide step, measured slower: 33.5 against 27.8 us for ViT-L qkv.)
 template <int LOG2B, int BITS, int NT>
 __device__ __forceinline__ void fuse_act_worker(int at, const __half *__restrict__ X, int64_t M, int K,
                                                 int8_t *Xq, float *x_scale, unsigned int *counters,

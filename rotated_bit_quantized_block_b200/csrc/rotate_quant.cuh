@@ -407,6 +407,24 @@ __device__ __forceinline__ void act_store_codes(float2 (&bv)[8][2], float fac1, 
     }
 }
 
+// Packed int4 weight codes (a byte holds element 2j in its low nibble and
+// 2j+1 in its high nibble, two's complement) to one int8 code per byte, in
+// element order: 16 packed bytes in, 32 code bytes out.
+__device__ __forceinline__ void widen_int4_to_int8(uint4 p, uint4 &out0, uint4 &out1) {
+    const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        // sign-extend each nibble within its byte: (n ^ 8) - 8, bytewise
+        const uint32_t lo = __vsub4((w[i] & 0x0f0f0f0fu) ^ 0x08080808u, 0x08080808u);
+        const uint32_t hi = __vsub4(((w[i] >> 4) & 0x0f0f0f0fu) ^ 0x08080808u, 0x08080808u);
+        o[2 * i] = __byte_perm(lo, hi, 0x5140);
+        o[2 * i + 1] = __byte_perm(lo, hi, 0x7362);
+    }
+    out0 = make_uint4(o[0], o[1], o[2], o[3]);
+    out1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
 // BITS fixes the code range (8: [-127, 127], 4: [-8, 7]); PACKED stores int4
 // codes two per byte, otherwise every code takes one byte.
 // One CTA handles `rows` consecutive rows with L = K/32 threads each (the
@@ -417,7 +435,9 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
                                                                 int rows, void *__restrict__ Xq,
                                                                 float *__restrict__ x_scale,
                                                                 uint4 *__restrict__ zero16,
-                                                                int64_t n_zero16) {
+                                                                int64_t n_zero16,
+                                                                const uint4 *__restrict__ w_packed,
+                                                                uint4 *__restrict__ w_wide, int64_t n_w16) {
     extern __shared__ __align__(16) uint8_t act_smem[];
     __shared__ unsigned int s_amax[kMaxRowsPerCta];
     __shared__ float s_fac[kMaxRowsPerCta];
@@ -446,6 +466,15 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + tid; i < n_zero16;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)
         zero16[i] = make_uint4(0u, 0u, 0u, 0u);
+    // the W4A4 linear's packed int4 weights, widened once to int8 codes for the
+    // GEMM that follows (n_w16 units of 16 packed bytes)
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + tid; i < n_w16;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        uint4 o0, o1;
+        widen_int4_to_int8(ld_stream_v4(w_packed + i), o0, o1);
+        w_wide[2 * i] = o0;
+        w_wide[2 * i + 1] = o1;
+    }
     if (tid < rows) s_amax[tid] = 0u;
     float2 a[4][4];
     act_layout_a<LOG2B>(raw, false, a);

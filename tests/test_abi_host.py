@@ -127,9 +127,11 @@ def test_linear_workspace_bytes_adds_split_k_room(lib):
     # token-major stream-K (deep K, a partly filled last round of 128 x 256 tiles):
     # one 128 x 256 int32 partial-tile slot per boundary between the 148 shares (+1)
     slots = 149 * 128 * 256 * 4
-    assert lws(5184, 4096, 1024, 4) == ws(5184, 4096, 4) + 2048 + slots
-    for bits in (8, 4):
-        assert lws(2500, 8192, 2000, bits) == ws(2500, 8192, bits) + 2048 + slots
+    assert lws(2500, 8192, 2000, 8) == ws(2500, 8192, 8) + 2048 + slots
+    # W4A4 over more than 128 tokens: the int8-weight plan's split state, then
+    # the weights widened to one int8 code per byte (N x K)
+    assert lws(2500, 8192, 2000, 4) == ws(2500, 8192, 4) + 2048 + slots + 2000 * 8192
+    assert lws(5184, 4096, 1024, 4) == ws(5184, 4096, 4) + 2048 + 1024 * 4096
     # shallow K (the shared tiles cost more than the idle SMs): whole tiles, counters only
     for K, N in [(1024, 3072), (1024, 1024), (1024, 4096)]:
         assert lws(5184, K, N, 8) == ws(5184, K, 8) + 2048

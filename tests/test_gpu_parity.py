@@ -498,3 +498,36 @@ def test_linear_reads_weights_written_just_before(M, N, K, bits):
     assert np.array_equal(y_chained.view(np.uint16), y_after.view(np.uint16))
     # and the weights really changed: the zero codes give bias-only rows
     assert not np.array_equal(y_after.view(np.uint16), np.broadcast_to(bias.astype(np.float16), y_after.shape).view(np.uint16))
+
+
+@pytest.mark.parametrize("M,N,K", [(5184, 3072, 1024), (700, 1000, 4096), (129, 264, 128)])
+def test_w4a4_linear_widens_weights_once(M, N, K):
+    """W4A4 over more than 128 tokens with the linear workspace: the activation
+    launch widens the packed int4 weights once to int8 codes in the workspace
+    (after the int8-weight plan's part) and the int8-weight GEMM multiplies
+    them.  The widened codes equal the oracle's unpacking, and the output
+    equals the linear that widens tiles in shared memory (minimum workspace)
+    and the oracle's GEMM of the workspace's codes, bit for bit."""
+    X = wl.activations(M, K, 0.01, 30.0, seed=M)
+    W = wl.weight(N, K, 0.02, seed=N)
+    bias = wl.bias(N, seed=K)
+    Xd, bd = dev(X), dev(bias)
+    Wq, sw = cr.convrot_quantize_weight(dev(W), 128, 4, cr.CLIP_MSE)
+    big = cr.convrot_linear_workspace_bytes(M, K, N, 4)
+    assert cr.convrot_linear_plan(M, K, N, 4, 128, big)["weights_widened"] == 1
+    ws = torch.empty(big, dtype=torch.uint8, device="cuda")
+    y = host(cr.convrot_linear_w4a4(Xd, Wq, sw, 128, bias=bd, workspace=ws))
+    raw = host(ws)
+    off = cr.convrot_linear_workspace_bytes(M, K, N, 8)
+    wide = raw[off: off + N * K].view(np.int8).reshape(N, K)
+    qw = oracle.unpack_int4(host(Wq))
+    assert np.array_equal(wide, qw)
+    ws_small = torch.empty(cr.convrot_workspace_bytes(M, K, 4), dtype=torch.uint8, device="cuda")
+    y_small = host(cr.convrot_linear_w4a4(Xd, Wq, sw, 128, bias=bd, workspace=ws_small))
+    assert np.array_equal(y.view(np.uint16), y_small.view(np.uint16))
+    qx = raw[: M * K].view(np.int8).reshape(M, K)
+    o = (M * K + 255) // 256 * 256
+    sx = raw[o: o + 4 * M].view(np.float32)
+    rows = np.unique(np.linspace(0, M - 1, 33).astype(int))
+    yr = oracle.gemm_dequant(qx[rows], sx[rows], qw, host(sw), bias)
+    assert np.array_equal(y[rows].view(np.uint16), yr.view(np.uint16))

@@ -31,12 +31,12 @@ def test_abandoned_wait_reports_timeout_once(kind):
     r = result.cpu().numpy()
     assert r[0] == 0 and r[1] == 1
     cr.convrot_device_status()  # reported once, then cleared
-    # the context is usable: a fused linear equals the two-launch linear
+    # the context is usable: the fused linear equals the two-launch linear
     M, N, K = 640, 1024, 1024
     X = torch.from_numpy(wl.activations(M, K, 0.01, 30.0, seed=kind)).cuda()
     W = torch.from_numpy(wl.weight(N, K, 0.02, seed=kind + 1)).cuda()
     Wq, sw = cr.convrot_quantize_weight(W, 128, 8, cr.CLIP_MSE)
-    y1 = cr.convrot_linear_w8a8(X, Wq, sw, 128)
+    y1 = cr.convrot_linear_w8a8_fused(X, Wq, sw, 128)
     ws = torch.empty(cr.convrot_workspace_bytes(M, K, 8), dtype=torch.uint8, device="cuda")
     cr.convrot_linear_quant_act(X, 128, 8, ws)
     y2 = cr.convrot_linear_gemm(ws, M, K, 8, Wq, sw)
