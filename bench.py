@@ -577,7 +577,7 @@ def ours_arm(args, w, rank, world, local_rank):
 
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    n_sets = set_count(w)
+    n_sets = args.sets if args.sets > 0 else set_count(w)
     reps = [Replica(w, replica=r, device=device, host_copies=True) for r in replica_ids(rank, n_sets)]
     torch.cuda.synchronize()
     setup_s = time.perf_counter() - t0
@@ -642,8 +642,11 @@ def ours_arm(args, w, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": dtype_of(w), "data": "synthetic",
-        "config": dict(config_of(w), l2=f"inputs larger than L2: {n_sets} rotating buffer sets of "
-                                        f"{per_set / 2**20:.0f} MiB each (L2 {L2_BYTES >> 20} MiB)"),
+        "config": dict(config_of(w), l2=(f"inputs larger than L2: {n_sets} rotating buffer sets of "
+                                         f"{per_set / 2**20:.0f} MiB each (L2 {L2_BYTES >> 20} MiB)"
+                                         if n_sets * per_set > 1.5 * L2_BYTES else
+                                         f"{n_sets} buffer set(s) of {per_set / 2**20:.0f} MiB: "
+                                         f"NOT larger than 1.5 x L2 (profiling run)")),
         "tops": m["tops"] * world,
         "roofline": roofline,
         "rotate_quant": rotate_quant,
@@ -723,6 +726,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub-results", action="store_true")
     ap.add_argument("--sub-steps", type=int, default=10)
+    # rotating buffer sets (default: enough to move 1.5 x L2 per pass); fewer
+    # only to keep a profiler capture small -- its timings then see warm L2
+    ap.add_argument("--sets", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -154,11 +154,11 @@ void rotate_geometry(int64_t K, int *rows, int *threads) {
 // wave is launched as exactly one wave (a partial second wave would repeat the
 // whole load-compute-store latency).
 template <typename Kern>
-void act_geometry(Kern kernel, int sms, int64_t M, int64_t K, int *rows, int *threads) {
+void act_geometry(Kern kernel, int sms, int64_t M, int64_t K, int *rows, int *threads, int *resident) {
     const int L = static_cast<int>(K / convrot::kElemsPerThread);
     int R0, T0;
     rotate_geometry(K, &R0, &T0);
-    int best_R = R0, best_T = T0;
+    int best_R = R0, best_T = T0, best_cap = 0;
     int64_t best_cost = -1;
     const int rmax_threads = 1024 / L;
     const int r_hi = rmax_threads < convrot::kMaxRowsPerCta ? rmax_threads : convrot::kMaxRowsPerCta;
@@ -179,10 +179,12 @@ void act_geometry(Kern kernel, int sms, int64_t M, int64_t K, int *rows, int *th
             best_cost = cost;
             best_R = R;
             best_T = T;
+            best_cap = static_cast<int>(cap);
         }
     }
     *rows = best_R;
     *threads = best_T;
+    *resident = best_cap;  // CTAs of this geometry the GPU holds at once (0: unknown)
 }
 
 // Launches with programmatic stream serialization: the kernel may begin while
@@ -250,12 +252,14 @@ void launch_act(const void *X, int64_t M, int64_t K, void *Xq, float *xs, cudaSt
             configured[dev] = true;
         }
     }
-    int R, T;
-    act_geometry(kern, sms, M, K, &R, &T);
+    int R, T, resident;
+    act_geometry(kern, sms, M, K, &R, &T, &resident);
     const int64_t grid = (M + R - 1) / R;
+    // a grid of more than one wave prefetches one wave ahead
+    const int pf_ahead = (resident > 0 && grid > resident) ? resident : 0;
     launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(T), static_cast<size_t>(convrot::act_smem_bytes(T)), st,
                static_cast<const __half *>(X), M, static_cast<int>(K), R, Xq, xs, ex.zero16, ex.n_zero16, ex.w_packed,
-               ex.w_wide, ex.n_w16);
+               ex.w_wide, ex.n_w16, pf_ahead);
 }
 
 template <int BITS, bool PACKED>
