@@ -132,26 +132,21 @@ convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, i
 size_t convrot_workspace_bytes(int64_t M, int64_t K, int bits);
 
 /*
- * Workspace size that also lets the linear split the K loop of its GEMM across
- * SMs.  For the fewest tokens (M <= 4 with int8 weights, M <= 8 with int4) the
- * GEMM is a weight-streaming kernel that needs no split.  Up to M = 128 it
- * runs feature-major (128 output features x 32 tokens per tile) and has too
- * few tiles to fill the GPU; with this
- * workspace the K slices of a tile run on separate SMs and add their int32
- * partials into an M x N buffer.  For more tokens, where the 128 x 256 output
- * tiles fill some but not all SMs in their last round (and CTA pairs are not
- * used), the GEMM runs stream-K: every SM takes an equal share of all tiles'
- * K steps, and a tile shared by two SMs is summed from one int32 partial tile
- * (128 x 256) that the first of them stores in a slot of this workspace.
- * Size: convrot_workspace_bytes(M, K, bits) plus 2 KB of split-K counters plus
- * that buffer (rounded up to 256 bytes) or (SMs + 1) partial-tile slots of
- * 128 KB.  For W4A4 over more than 128 tokens it also holds the weights
- * widened to int8 codes (N*K bytes, after the split buffer of the int8-weight
- * plan): see convrot_linear_w4a4.  The activation half of the linear zeroes the counters and the M x N
- * buffer; the GEMM half leaves both zeroed again (the partial-tile slots are
- * written before they are read and need no zeroing).  With only the minimum
- * workspace the linears never split.  Depends on the current device's SM
- * count.  Returns 0 for invalid arguments.
+ * Workspace size that also lets the linear balance its GEMM across SMs.  For
+ * more than 128 tokens, where the 128 x 256 output tiles fill some but not all
+ * SMs in their last round (and CTA pairs are not used), the GEMM runs
+ * stream-K: every SM takes an equal share of all tiles' K steps, and a tile
+ * shared by two SMs is summed from one int32 partial tile (128 x 256) that the
+ * first of them stores in a slot of this workspace.  (With at most 128 tokens
+ * the GEMM splits K over clusters of CTAs that add their partials through
+ * distributed shared memory, which needs no workspace.)
+ * Size: convrot_workspace_bytes(M, K, bits) plus 2 KB of counters plus, where
+ * stream-K applies, (SMs + 1) partial-tile slots of 128 KB.  For W4A4 over
+ * more than 128 tokens it also holds the weights widened to int8 codes (N*K
+ * bytes, after the slots of the int8-weight plan): see convrot_linear_w4a4.
+ * The activation half of the linear zeroes the counters; the GEMM half leaves
+ * them zeroed again (the partial-tile slots are written before they are read).
+ * Depends on the current device's SM count.  Returns 0 for invalid arguments.
  */
 size_t convrot_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits);
 
@@ -164,7 +159,7 @@ size_t convrot_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int bits)
  *   bias      [N] fp16 or NULL.
  *   Y         [M x N] fp16 output.
  *   workspace at least convrot_workspace_bytes(M, K, 8) bytes of device memory
- *             (convrot_linear_workspace_bytes(M, K, N, 8) enables split-K); on
+ *             (convrot_linear_workspace_bytes(M, K, N, 8) enables stream-K); on
  *             return it holds the activation codes (int8 M x K) followed, at the
  *             next 256-byte boundary, by the scales.
  */
@@ -195,7 +190,9 @@ convrot_status_t convrot_linear_w4a4(const void *X, int64_t M, int64_t K, const 
  *              features); 1: feature-major tiles (128 features x tile_n
  *              tokens); 2: the weight-streaming kernel (dp4a).
  *   cta_pair / stream_k / k_splits: CTA pairs (cta_group::2), stream-K shares,
- *              K slices of the feature-major split.
+ *              K slices of the feature-major split (a cluster of that many
+ *              CTAs per tile; fewer at launch if the GPCs cannot hold all the
+ *              clusters at once).
  *   fused_available  1 if convrot_linear_w8a8_fused accepts the call (W8A8).
  *   weights_widened  1 if the W4A4 linear widens its weights to int8 codes in
  *              the workspace and runs the int8-weight GEMM (the fields above
@@ -242,10 +239,9 @@ convrot_status_t convrot_linear_w8a8_fused(const void *X, int64_t M, int64_t K, 
  * The two launches of convrot_linear_w8a8 / convrot_linear_w4a4, callable
  * separately (same arguments, same workspace layout): first rotate and
  * quantize X into the workspace, then run the integer GEMM + dequant from it.
- * The workspace must not be reused by another linear in between.  Not knowing
- * N, convrot_linear_quant_act zeroes everything after the scales (for M <= 128
- * at most the split state of a GEMM with N <= 32768; for larger M only the
- * counters).
+ * The workspace must not be reused by another linear in between.
+ * convrot_linear_quant_act zeroes the 2 KB of counters after the scales where
+ * the workspace holds them.
  */
 convrot_status_t convrot_linear_quant_act(const void *X, int64_t M, int64_t K, int block, int bits,
                                           void *workspace, size_t workspace_bytes, void *stream);

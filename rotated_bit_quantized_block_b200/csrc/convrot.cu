@@ -340,8 +340,7 @@ constexpr int kMaxSplitTiles = 512;              // split-K counters in a linear
 constexpr size_t kCounterBytes = kMaxSplitTiles * 4;
 static_assert(kCounterBytes == convrot::kFuseMaxPanels * 4, "the fused linear's panel counters fill the counter area");
 constexpr int64_t kSwapMaxTokens = 128;          // feature-major up to this many tokens
-constexpr int kSwapTokens = 32;                  // token tile of the feature-major GEMM
-constexpr int64_t kMaxSplitFeatures = 32768;     // split K only for N up to this
+constexpr int kMinSliceSteps = 4;                // K steps of 128 in a feature-major split-K slice
 // Stream-K: the cost of the shared tiles (148 partial tiles of 128 KB stored and
 // read back, ~5 us on B200), in 128-deep steps of a 256-wide tile: int8 weights
 // / widened int4 weights (whose steps are slower).  Measured, CUDA-graph-timed,
@@ -350,29 +349,28 @@ constexpr int64_t kMaxSplitFeatures = 32768;     // split K only for N up to thi
 constexpr double kStreamKOverheadSteps8 = 16.0;
 constexpr double kStreamKOverheadSteps4 = 9.0;
 
-// Few tokens: feature-major tiles (128 features x 32 tokens), K split so that
-// the tiles x splits units cover the SMs (at most 8 slices, each at least 8
-// K steps of 128: a split costs a few microseconds of counting and re-reading,
-// which shorter slices do not repay).  Otherwise token-major 128 x 256 tiles,
-// narrowed to 128 when 256-wide tiles would leave more than half the SMs idle.
-// (Measured on B200 with CUDA-graph launches: feature-major wins up to 128
-// tokens, token-major from 192.)
+// Few tokens: feature-major tiles of 128 features x all the tokens (32, 64 or
+// 128 columns), so that every weight byte is read once.  Where the tiles alone
+// leave SMs idle, K is split over a cluster of 2, 4 or 8 CTAs (each slice at
+// least kMinSliceSteps steps of 128), whose partial accumulators are added
+// through distributed shared memory.  Otherwise token-major 128 x 256 tiles,
+// narrowed when narrower tiles finish in fewer rounds.  (Measured on B200 with
+// CUDA-graph launches: feature-major wins up to 128 tokens, token-major from 192.)
 GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split, bool w4 = false) {
     GemmPlan p;
     if (M <= kSwapMaxTokens) {
         p.swap = true;
-        p.bn = kSwapTokens;
-        p.tiles = ((N + 127) / 128) * ((M + p.bn - 1) / p.bn);
+        p.bn = M <= 32 ? 32 : (M <= 64 ? 64 : 128);
+        p.tiles = (N + 127) / 128;
         // for the fewest tokens the weight-streaming kernel runs instead (int8
         // activation codes; the feature-major tiles stay for packed ones).
         // Measured on B200 (K = N = 4096, CUDA graphs): faster up to 4 tokens
         // with int8 weights (4.9 against 8.2 us at M = 1), up to 8 with int4
         p.gemv = M <= (w4 ? 8 : 4);
-        if (allow_split && !p.gemv && p.tiles > 0 && p.tiles <= kMaxSplitTiles && N <= kMaxSplitFeatures) {
-            int64_t s = sms / p.tiles;
-            if (s > 8) s = 8;
-            if (s > K / 1024) s = K / 1024;
-            if (s >= 2) p.splits = static_cast<int>(s);
+        if (!p.gemv) {
+            int s = 8;
+            while (s > 1 && (p.tiles * s > sms || K / 128 < static_cast<int64_t>(s) * kMinSliceSteps)) s /= 2;
+            p.splits = s;
         }
         return p;
     }
@@ -420,11 +418,12 @@ GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split, b
     return p;
 }
 
-// int32 M x N sum buffer of a split feature-major GEMM, or the partial-tile
-// slots of a stream-K one (one 128 x BN int32 tile per boundary between CTAs).
+// The partial-tile slots of a stream-K GEMM (one 128 x BN int32 tile per
+// boundary between CTAs; a feature-major split-K GEMM needs no global state).
 size_t split_buffer_bytes(const GemmPlan &p, int64_t M, int64_t N) {
-    if (p.streamk > 0) return static_cast<size_t>(p.streamk + 1) * 128 * p.bn * 4;
-    return p.splits > 1 ? round256(static_cast<size_t>(M) * N * 4) : 0;
+    (void)M;
+    (void)N;
+    return p.streamk > 0 ? static_cast<size_t>(p.streamk + 1) * 128 * p.bn * 4 : 0;
 }
 
 // The fused linear's activation input: the fp16 X, its block size and the
@@ -460,7 +459,8 @@ template <class Cfg, int FL = -1, int FB = 8>
 convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, const void *Wc, int64_t M, int64_t N,
                                  int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
                                  int32_t *acc_out, cudaStream_t st, int splits, int32_t *acc_buf,
-                                 unsigned int *counters, int streamk = 0, const FusePrologue *fuse = nullptr) {
+                                 unsigned int *counters, int streamk = 0, const FusePrologue *fuse = nullptr,
+                                 bool w_early = true) {
     const auto kern = convrot::gemm_i8_tcgen05_kernel<Cfg, FL, FB>;
     const __half *fx = fuse ? static_cast<const __half *>(fuse->X) : nullptr;
     int8_t *fq = fuse ? static_cast<int8_t *>(const_cast<void *>(Xc)) : nullptr;
@@ -489,8 +489,38 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, cons
     CR_TRY(op_map(&tb, Cfg::SWAP ? Xc : Wc, rows_b, Cfg::B_ROWS, Cfg::B4));
     if (Cfg::SWAP) ty = ta;  // stores go straight to Y
     else CR_TRY(make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
-    const int64_t units =
-        ((rows_a + Cfg::TILE_M - 1) / Cfg::TILE_M) * ((rows_b + Cfg::BN - 1) / Cfg::BN) * splits;
+    const int64_t tiles = ((rows_a + Cfg::TILE_M - 1) / Cfg::TILE_M) * ((rows_b + Cfg::BN - 1) / Cfg::BN);
+    if (Cfg::SWAP && splits > 1) {
+        // the clusters of all tiles must be co-resident (one CTA per SM): fewer
+        // K slices where the GPCs cannot place that many clusters of this size
+        static std::mutex mu;
+        static int max_clusters[kMaxDevices][4] = {};  // by log2 of the cluster size
+        std::lock_guard<std::mutex> lock(mu);
+        while (splits > 1) {
+            const int lg = splits == 2 ? 1 : (splits == 4 ? 2 : 3);
+            int &mc = max_clusters[dev][lg];
+            if (mc == 0) {
+                cudaLaunchConfig_t occ = {};
+                occ.gridDim = dim3(static_cast<unsigned>(splits * (info->sms / splits)));
+                occ.blockDim = dim3(Cfg::NUM_THREADS);
+                occ.dynamicSmemBytes = Cfg::SMEM_BYTES;
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                occ.attrs = attr;
+                occ.numAttrs = 1;
+                int n = 0;
+                cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &occ);
+                if (e != cudaSuccess) cudaGetLastError();
+                mc = (e == cudaSuccess && n > 0) ? n : -1;
+            }
+            if (mc > 0 && tiles <= mc) break;
+            splits /= 2;
+        }
+    }
+    const int64_t units = tiles * splits;
     if (Cfg::PAIR) {
         // persistent: one cluster of two CTAs per co-resident pair of SMs
         static int max_clusters[kMaxDevices] = {};
@@ -520,14 +550,23 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, cons
         launch_pdl_cluster(kern, dim3(static_cast<unsigned>(2 * clusters)), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st,
                            2u, ta, tb, ty, static_cast<int>(rows_a), static_cast<int>(rows_b), static_cast<int>(K), sx,
                            sw, static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out, splits, acc_buf,
-                           counters, 0, fx, fq, fs, ff);
+                           counters, 0, fx, fq, fs, ff, w_early ? 1 : 0);
         return launch_status("gemm_i8_tcgen05 (CTA pairs)");
+    }
+    if (Cfg::SWAP && splits > 1) {
+        // split K: one CTA per (tile, K slice), the slices of a tile in one cluster
+        launch_pdl_cluster(kern, dim3(static_cast<unsigned>(units)), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st,
+                           static_cast<unsigned>(splits), ta, tb, ty, static_cast<int>(rows_a),
+                           static_cast<int>(rows_b), static_cast<int>(K), sx, sw, static_cast<const __half *>(bias),
+                           static_cast<__half *>(Y), acc_out, splits, acc_buf, counters, 0, fx, fq, fs, ff,
+                           w_early ? 1 : 0);
+        return launch_status("gemm_i8_tcgen05 (split-K clusters)");
     }
     // persistent: one CTA per SM (stream-K: exactly the planned number of shares)
     const int grid = streamk > 0 ? streamk : static_cast<int>(units < info->sms ? units : info->sms);
     launch_pdl(kern, dim3(grid), dim3(Cfg::NUM_THREADS), Cfg::SMEM_BYTES, st, ta, tb, ty, static_cast<int>(rows_a),
                static_cast<int>(rows_b), static_cast<int>(K), sx, sw, static_cast<const __half *>(bias),
-               static_cast<__half *>(Y), acc_out, splits, acc_buf, counters, streamk, fx, fq, fs, ff);
+               static_cast<__half *>(Y), acc_out, splits, acc_buf, counters, streamk, fx, fq, fs, ff, w_early ? 1 : 0);
     return launch_status("gemm_i8_tcgen05");
 }
 
@@ -590,34 +629,42 @@ template <bool X4, bool W4>
 convrot_status_t launch_gemm(DeviceInfo *info, int dev, const void *Xc, const void *Wc, int64_t M, int64_t N,
                              int64_t K, const float *sx, const float *sw, const void *bias, void *Y,
                              int32_t *acc_out, cudaStream_t st, const GemmPlan &p, int32_t *acc_buf = nullptr,
-                             unsigned int *counters = nullptr) {
+                             unsigned int *counters = nullptr, bool w_early = true) {
     using convrot::GemmCfg;
     if constexpr (!X4) {
         if (p.gemv) return launch_gemv<W4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
     }
-    if (p.swap)
-        return launch_gemm_cfg<GemmCfg<kSwapTokens, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y,
-                                                                   acc_out, st, p.splits, acc_buf, counters);
+    if (p.swap) {
+        if (p.bn == 32)
+            return launch_gemm_cfg<GemmCfg<32, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st,
+                                                              p.splits, nullptr, nullptr, 0, nullptr, w_early);
+        if (p.bn == 64)
+            return launch_gemm_cfg<GemmCfg<64, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st,
+                                                              p.splits, nullptr, nullptr, 0, nullptr, w_early);
+        return launch_gemm_cfg<GemmCfg<128, W4, X4, true>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st,
+                                                           p.splits, nullptr, nullptr, 0, nullptr, w_early);
+    }
     if constexpr (!X4) {  // (stream-K needs a linear's workspace, whose activation codes are bytes)
         if (p.streamk > 0)  // token-major, single CTAs, 256-wide tiles
             return launch_gemm_cfg<GemmCfg<256, false, W4, false, false, true>>(
-                info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1, acc_buf, counters, p.streamk);
+                info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1, acc_buf, counters, p.streamk, nullptr,
+                w_early);
     }
     if (p.bn == 192)
         return launch_gemm_cfg<GemmCfg<192, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
-                                                     nullptr, nullptr);
+                                                     nullptr, nullptr, 0, nullptr, w_early);
     if (p.bn == 256) {
         if constexpr (!X4 && !W4) {
             if (p.pair)
                 return launch_gemm_cfg<GemmCfg<256, false, false, false, true>>(info, dev, Xc, Wc, M, N, K, sx, sw,
                                                                                 bias, Y, acc_out, st, 1, nullptr,
-                                                                                nullptr);
+                                                                                nullptr, 0, nullptr, w_early);
         }
         return launch_gemm_cfg<GemmCfg<256, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1,
-                                                     nullptr, nullptr);
+                                                     nullptr, nullptr, 0, nullptr, w_early);
     }
     return launch_gemm_cfg<GemmCfg<128, X4, W4>>(info, dev, Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 1, nullptr,
-                                                 nullptr);
+                                                 nullptr, 0, nullptr, w_early);
 }
 
 convrot_status_t check_gemm_args(const void *Xq, const float *xs, int64_t M, const void *Wq, const float *ws,
@@ -823,21 +870,12 @@ static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int
     float *xs;
     unsigned int *counters;
     workspace_parts(workspace, M, K, &xq, &xs, &counters);
-    // the split-K counters and sum buffer that follow the codes and scales are
-    // zeroed here for the GEMM half
+    // the counters that follow the codes and scales are zeroed here for the
+    // GEMM half (stream-K's partial slots are written before they are read)
     const size_t base = convrot_workspace_bytes(M, K, bits);
     size_t zero_bytes = 0;
-    if (workspace_bytes > base) {
-        size_t cap;
-        if (n_features >= 0) {
-            // (stream-K partial slots are written before they are read: only the counters)
-            const GemmPlan p = plan_gemm(info->sms, M, n_features, K, true, bits == 4 && wide == nullptr);
-            cap = kCounterBytes + (p.streamk > 0 ? 0 : split_buffer_bytes(p, M, n_features));
-        } else {
-            cap = kCounterBytes + (M <= kSwapMaxTokens ? round256(static_cast<size_t>(M) * kMaxSplitFeatures * 4) : 0);
-        }
-        zero_bytes = (workspace_bytes - base < cap ? workspace_bytes - base : cap) & ~size_t(15);
-    }
+    if (workspace_bytes > base)
+        zero_bytes = (workspace_bytes - base < kCounterBytes ? workspace_bytes - base : kCounterBytes) & ~size_t(15);
     ActExtras ex;
     ex.zero16 = zero_bytes ? reinterpret_cast<uint4 *>(counters) : nullptr;
     ex.n_zero16 = static_cast<int64_t>(zero_bytes / 16);
@@ -850,12 +888,12 @@ static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int
     return rotate_quant_act_impl(X, M, K, block, bits, false, xq, xs, st, info->sms, dev, ex);
 }
 
-// The GEMM plan of a linear's second launch: split K only when the workspace
-// holds the counters and the sum buffer (which the activation half zeroed).
+// The GEMM plan of a linear's second launch: stream-K only when the workspace
+// holds the counters (which the activation half zeroed) and the partial slots.
 static GemmPlan two_launch_plan(int sms, int64_t M, int64_t N, int64_t K, int bits, size_t workspace_bytes) {
     GemmPlan p = plan_gemm(sms, M, N, K, true, bits == 4);
     const size_t base = convrot_workspace_bytes(M, K, bits) + kCounterBytes;
-    if ((p.splits > 1 || p.streamk > 0) && workspace_bytes < base + split_buffer_bytes(p, M, N))
+    if (p.streamk > 0 && workspace_bytes < base + split_buffer_bytes(p, M, N))
         p = plan_gemm(sms, M, N, K, false, bits == 4);
     return p;
 }
@@ -878,7 +916,7 @@ static bool fused_plan(int sms, int64_t M, int64_t K, int64_t N, int bits, int b
 
 static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace_bytes, int64_t M, int64_t K,
                                          int bits, const void *Wq, const float *w_scale, int64_t N,
-                                         const void *bias, void *Y, cudaStream_t st) {
+                                         const void *bias, void *Y, cudaStream_t st, bool w_early = true) {
     CR_TRY(check_workspace(workspace, workspace_bytes, M, K, bits));
     void *xq;
     float *xs;
@@ -892,9 +930,9 @@ static convrot_status_t linear_gemm_impl(const void *workspace, size_t workspace
     const GemmPlan p = two_launch_plan(info->sms, M, N, K, bits, workspace_bytes);
     if (bits == 8)
         return launch_gemm<false, false>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st, p, acc_buf,
-                                         counters);
+                                         counters, w_early);
     return launch_gemm<false, true>(info, dev, xq, Wq, M, N, K, xs, w_scale, bias, Y, nullptr, st, p, acc_buf,
-                                    counters);
+                                    counters, w_early);
 }
 
 static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t K, const void *Wq,
@@ -915,7 +953,8 @@ static convrot_status_t linear_impl(int bits, const void *X, int64_t M, int64_t 
             // the activation launch also widens the weights; the int8-weight GEMM follows
             CR_TRY(linear_act_impl(X, M, K, block, 4, workspace, workspace_bytes, st, N, Wq));
             const int8_t *wide = static_cast<const int8_t *>(workspace) + off;
-            return linear_gemm_impl(workspace, workspace_bytes, M, K, 8, wide, w_scale, N, bias, Y, st);
+            // (the widened weights come from the activation launch: no early prefetch)
+            return linear_gemm_impl(workspace, workspace_bytes, M, K, 8, wide, w_scale, N, bias, Y, st, false);
         }
     }
     CR_TRY(linear_act_impl(X, M, K, block, bits, workspace, workspace_bytes, st, N));

@@ -141,6 +141,14 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Prefetches one box of a 2D tensor map into L2 (a hint: no data reaches the
+// SM and no later load can see stale values through it).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
 // 2D tiled bulk copy global -> shared (no multicast), completing on `bar`.
 // x is the innermost coordinate (bytes for the 8-bit maps used here; always
 // a multiple of 64), y the row coordinate.
@@ -280,6 +288,52 @@ __device__ __forceinline__ void cluster_sync() {
 // Arrive on an mbarrier given by its shared::cluster address (possibly the peer's).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+
+// Bounded wait (every lane of the warp) for a phase completed by arrivals from
+// other CTAs of the cluster: acquire at cluster scope, so that what those CTAs'
+// threads wrote to their own shared memory before arriving (release, cluster
+// scope) is visible to this warp's distributed-shared-memory loads.
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    bool ok = true;
+    if (!mbar_try_wait_acq_cluster(bar, parity)) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_acq_cluster(bar, parity)) {
+            if (*abort) {
+                ok = false;
+                break;
+            }
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(&g_device_status, kStatusTimeout);
+                *abort = 1;
+                ok = false;
+                break;
+            }
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+// 16-byte load from the shared memory of a CTA of the cluster (shared::cluster address).
+__device__ __forceinline__ uint4 ld_dsmem_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
 }
 
 // TMA load into this CTA's shared memory whose completion is counted on the

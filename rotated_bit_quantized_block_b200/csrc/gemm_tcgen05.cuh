@@ -26,13 +26,15 @@
 //     B = weight codes (BN output features); the epilogue stages 32 x 32 fp16
 //     boxes in shared memory and writes them with TMA stores.
 //   * feature-major (SWAP = true, few tokens): A = weight codes (128 output
-//     features per tile), B = activation codes (BN tokens, e.g. 32), so
-//     the tensor core is not spent on empty token rows and the weights stream
-//     through a deep ring.  Each epilogue thread owns one output feature and
-//     writes token columns with coalesced stores.  The K loop may be split
-//     across CTAs: every slice adds its int32 partial into a zeroed M x N
-//     buffer (red.add), and the slice that counts in last dequantizes the sum
-//     and zeroes the buffer again.
+//     features per tile), B = activation codes (BN = 32, 64 or 128 tokens:
+//     all of them, so every weight byte is read once), so the tensor core is
+//     not spent on empty token rows and the weights stream through a deep
+//     ring.  Each epilogue thread owns one output feature and writes token
+//     columns with coalesced stores.  The K loop may be split over a cluster
+//     of 2, 4 or 8 CTAs (one K slice each): the partial accumulators are added
+//     through distributed shared memory, each CTA summing and storing the
+//     pieces of some of its epilogue warps -- no global partials, counters or
+//     zeroing.
 //
 // Fused linear (Cfg::FUSE, token-major): the kernel also rotates and
 // quantizes the activations.  ACT_WARPS extra warps per CTA (register-fed, no
@@ -117,7 +119,10 @@ struct GemmCfg {
     static constexpr int ACT_MAX_K = ACT_THREADS * kElemsPerThread;  // a row fits the activation warps once
     static constexpr int ACT_SMEM_BYTES = FUSE ? 2 * (ACT_THREADS / 4) * 4 : 0;  // row-segment maxima, 2 units
     static constexpr int NUM_THREADS = 32 * (FIRST_ACT_WARP + ACT_WARPS);
-    static constexpr int FIXED_BARRIERS = 2 * PSTAGES + 4 + 1 + 2 + 2;
+    static constexpr int FIXED_BARRIERS = 2 * PSTAGES + 4 + 1 + 2 + 2 + 1;
+    // feature-major split K: an epilogue warp's piece of the accumulator (32
+    // TMEM lanes x EPI_COLS int32), exchanged through the idle MMA ring
+    static constexpr int PIECE_BYTES = 32 * EPI_COLS * 4;
     // MMA ring depth: as many stages as fit in the shared-memory budget (at most 12)
     static constexpr int SMEM_LIMIT = 232448;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - PSTAGES * PSTAGE_BYTES - OUT_BYTES - SCALE_BYTES -
@@ -136,7 +141,8 @@ struct GemmCfg {
     static_assert(SWAP ? (BN == 32 || BN == 64 || BN == 128 || BN == 256) : (BN % 64 == 0 && BN >= 64 && BN <= 256),
                   "tile width");
     static_assert(TMEM_COLS >= 2 * BN, "accumulators fit the allocation");
-    static_assert(EPI_COLS % CHUNK == 0, "epilogue chunking");
+    static_assert(EPI_COLS % CHUNK == 0 && CHUNK % 4 == 0, "epilogue chunking");
+    static_assert(!SWAP || EPI_WARPS * PIECE_BYTES <= STAGES * STAGE_BYTES, "split-K pieces fit the ring");
 };
 
 // Sign-extends 16 packed int4 codes (8 bytes, low nibble = even element) to 16
@@ -335,17 +341,22 @@ __global__ void abandoned_wait_kernel(int kind, uint64_t limit_ns, int32_t *resu
     result[1] = abort;
 }
 
+// Weight boxes a feature-major CTA prefetches into L2 before its grid-dependency wait.
+constexpr int kMaxEarlyBoxes = 64;
+
 // Kernel arguments, in the MMA's terms: the accumulator is M x N (rows of A x
 // rows of B).  Token-major: M = tokens, N = output features.  Feature-major:
 // M = output features, N = tokens.  sx is always the per-token scale, sw the
 // per-feature scale, bias per feature; Y and acc_out are tokens x features.
-// acc_buf / counters: the feature-major split-K sum buffer (M x N int32) and
-// per-tile counters; with streamk (Cfg::SK) the partial-tile slots (TILE_M x BN
-// int32 per CTA boundary) and per-boundary arrival counts (counters[b]) and
-// ready flags (counters[kStreamKFlags + b]).
+// splits > 1 (feature-major): the K slices of a tile, one CTA each, launched
+// as a cluster of `splits` CTAs.  acc_buf / counters (stream-K, Cfg::SK): the
+// partial-tile slots (TILE_M x BN int32 per CTA boundary), per-boundary
+// arrival counts (counters[b]) and ready flags (counters[kStreamKFlags + b]).
 // Fused linear (Cfg::FUSE; block 2^FLOG2B, activation codes one byte each in
 // the range of FBITS): X is the fp16 input, qx_out / sx_out the workspace that
 // tmA and sx cover, panels the zeroed panel counters (see above).
+// w_early != 0: the weight codes are not written by the previous kernel in the
+// stream, so their first tiles may be prefetched before the dependency wait.
 template <class Cfg, int FLOG2B = -1, int FBITS = 8>
 __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -353,7 +364,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                            const float *__restrict__ sw, const __half *__restrict__ bias, __half *__restrict__ Y,
                            int32_t *__restrict__ acc_out, int splits, int32_t *__restrict__ acc_buf,
                            unsigned int *__restrict__ counters, int streamk, const __half *__restrict__ X,
-                           int8_t *qx_out, float *sx_out, unsigned int *panels) {
+                           int8_t *qx_out, float *sx_out, unsigned int *panels, int w_early) {
     constexpr bool FUSED = Cfg::FUSE;
     static_assert(FUSED == (FLOG2B >= 0), "the activation warps need the block size");
     constexpr int BM = Cfg::BM, BN = Cfg::BN, STAGES = Cfg::STAGES, PSTAGES = Cfg::PSTAGES;
@@ -376,8 +387,9 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     uint64_t *scale_ready = drain + 1;                             // tile scales staged in smem
     uint64_t *scale_free = scale_ready + 1;                        // tile scales no longer read
     uint64_t *partial_done = scale_free + 1;                       // split K: this slice's partial added
-    uint64_t *decided = partial_done + 1;                          // split K: last-slice decision made
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(decided + 1);
+    uint64_t *decided = partial_done + 1;                          // stream-K: role decision made
+    uint64_t *red_in = decided + 1;                                // cluster split K: peers' pieces ready
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(red_in + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *s_last = reinterpret_cast<volatile int *>(tmem_slot + 2);
 
@@ -390,7 +402,13 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     const bool leader = rank == 0;
     const int first_unit = Cfg::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int unit_stride = Cfg::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
-    // split K (feature-major only): work unit u is K slice (u % splits) of tile (u / splits)
+    // split K (feature-major only): work unit u is K slice (u % splits) of tile (u / splits).
+    // The host launches one CTA per unit in clusters of `splits` CTAs (a tile's
+    // slices), which add their partial accumulators through distributed shared
+    // memory: the CTA of rank r sums and stores the pieces of the epilogue warps
+    // w with w % splits == r.
+    const bool csplit = Cfg::SWAP && splits > 1;
+    const uint32_t crank = csplit ? cluster_ctarank() : 0u;
     const int num_units = num_tiles * splits;
     auto unit_tile = [&](int u) { return u / splits; };
     auto unit_kb0 = [&](int u) { return (u - (u / splits) * splits) * num_kb / splits; };
@@ -445,6 +463,8 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
         mbar_init(scale_free, 32 * Cfg::EPI_WARPS);
         mbar_init(partial_done, 32 * Cfg::EPI_WARPS);
         mbar_init(decided, 1);
+        // every lane of the S - 1 other CTAs' warps whose pieces this CTA sums
+        mbar_init(red_in, csplit ? static_cast<uint32_t>((Cfg::EPI_WARPS / splits) * (splits - 1) * 32) : 1u);
         *abort = 0;
         fence_mbarrier_init();
     }
@@ -464,9 +484,26 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     }
     tc_fence_before_sync();
     __syncthreads();
-    if (Cfg::PAIR) cluster_sync();  // the peer's barriers are initialised before any remote use
+    if (Cfg::PAIR || csplit) cluster_sync();  // the peers' barriers are initialised before any remote use
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
+    // Weight codes that the previous kernel does not write (w_early): the first
+    // segment's weight tiles are prefetched into L2 while that kernel still runs
+    // (feature-major: the whole K slice, the few-token GEMM's entire stream;
+    // token-major: one ring's worth).
+    if (w_early != 0 && threadIdx.x == 0) {
+        const Seg g = seg_first();
+        if (g.tile >= 0) {
+            const int tm = g.tile / tiles_n, tn = g.tile - tm * tiles_n;
+            const int span = g.kb1 - g.kb0, cap = Cfg::SWAP ? kMaxEarlyBoxes : STAGES;
+            const int n = span < cap ? span : cap;
+            for (int i = 0; i < n; ++i) {
+                const int kb = g.kb0 + i;
+                if (Cfg::SWAP) tma_prefetch_l2_2d(&tmA, kb * (Cfg::A4 ? Cfg::BK / 2 : Cfg::BK), tm * BM);
+                else tma_prefetch_l2_2d(&tmB, kb * (Cfg::B4 ? Cfg::BK / 2 : Cfg::BK), tn * BN + rank * Cfg::B_ROWS);
+            }
+        }
+    }
     pdl_wait();  // the codes, scales and split-K buffers may come from the previous kernel
     pdl_launch_dependents();
     [[maybe_unused]] const int act_rpr = FUSED ? fuse_unit_rows(Cfg::ACT_THREADS, K) : 1;
@@ -652,7 +689,7 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
             load_scales(g0.tile >= 0 ? g0.tile : num_tiles, next_w, next_b);
         }
         int local = 0;
-        int n_split_units = 0;  // split units / shared tiles handled so far (parity of `decided`)
+        int n_split_units = 0;  // stream-K shared tiles handled so far (parity of `decided`)
         int n_partials = 0;     // stream-K partial tiles stored so far (parity of `partial_done`)
         for (Seg g = seg_first(); g.tile >= 0; g = seg_next(g), ++local) {
             const int tile = g.tile;
@@ -803,6 +840,16 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                 const float swf = row_ok ? sw[f] : 0.0f;
                 const float bf = (row_ok && bias != nullptr) ? __half2float(bias[f]) : 0.0f;
                 const int tok_base = tn * BN + cg * Cfg::EPI_COLS;
+                // Split K: a warp whose piece another CTA of the cluster sums stores
+                // its partial in its slot of this CTA's ring (idle: this CTA's one
+                // unit is done) as [column / 4][lane][4] int32, then each lane
+                // arrives on the summing CTA's red_in (release, cluster scope).  The
+                // summing warp waits for those arrivals and adds the peers' partials
+                // to its own.  Integer addition is exact: the order does not matter.
+                const uint32_t owner_rank = csplit ? static_cast<uint32_t>(ew % splits) : 0u;
+                const bool owner = owner_rank == crank;
+                uint8_t *piece = ring + ew * Cfg::PIECE_BYTES;
+                if (csplit && owner && !mbar_wait_cluster_warp(red_in, 0, abort)) break;
 #pragma unroll 1
                 for (int c = 0; c < NCHUNK; ++c) {
                     uint32_t r[CH];
@@ -813,60 +860,40 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
                         tc_fence_before_sync();
                         mbar_arrive(&tmem_empty[acc]);
                     }
+                    if (!owner) {
+#pragma unroll
+                        for (int j4 = 0; j4 < CH / 4; ++j4)
+                            *reinterpret_cast<uint4 *>(piece + ((c * (CH / 4) + j4) * 32 + lane) * 16) =
+                                make_uint4(r[4 * j4], r[4 * j4 + 1], r[4 * j4 + 2], r[4 * j4 + 3]);
+                        continue;
+                    }
+                    if (csplit) {
+                        for (int pr = 0; pr < splits; ++pr) {
+                            if (pr == static_cast<int>(crank)) continue;
+                            const uint32_t src = cluster_addr(piece, static_cast<uint32_t>(pr)) +
+                                                 static_cast<uint32_t>((c * (CH / 4) * 32 + lane) * 16);
+#pragma unroll
+                            for (int j4 = 0; j4 < CH / 4; ++j4) {
+                                const uint4 v = ld_dsmem_v4(src + j4 * 32 * 16);
+                                r[4 * j4] += v.x;
+                                r[4 * j4 + 1] += v.y;
+                                r[4 * j4 + 2] += v.z;
+                                r[4 * j4 + 3] += v.w;
+                            }
+                        }
+                    }
                     if (!row_ok) continue;
 #pragma unroll
                     for (int j = 0; j < CH; ++j) {
                         const int tok = tok_base + c * CH + j;
                         if (tok >= N) break;
                         const int64_t o = static_cast<int64_t>(tok) * M + f;
-                        if (splits > 1) {
-                            atomicAdd(acc_buf + o, static_cast<int32_t>(r[j]));  // result unused: a reduction
-                        } else {
-                            const int32_t a = static_cast<int32_t>(r[j]) >> Cfg::ACC_SHIFT;
-                            Y[o] = dequant1(a, col_s[cg * Cfg::EPI_COLS + c * CH + j], swf, bf);
-                            if (acc_out != nullptr) acc_out[o] = a;
-                        }
+                        const int32_t a = static_cast<int32_t>(r[j]) >> Cfg::ACC_SHIFT;
+                        Y[o] = dequant1(a, col_s[cg * Cfg::EPI_COLS + c * CH + j], swf, bf);
+                        if (acc_out != nullptr) acc_out[o] = a;
                     }
                 }
-                if (splits > 1) {
-                    __threadfence();  // this slice's additions are visible device-wide before it is counted
-                    mbar_arrive(partial_done);
-                    if (ew == 0 && lane == 0) {
-                        int last = 0;
-                        if (mbar_wait(partial_done, n_split_units & 1, abort)) {
-                            __threadfence();
-                            const unsigned int before = atomicAdd(&counters[tile], 1u);
-                            last = before == static_cast<unsigned int>(splits - 1);
-                            if (last) counters[tile] = 0u;  // ready for the next call
-                            __threadfence();               // the sum is read after the count
-                        }
-                        *s_last = last;
-                        mbar_arrive(decided);
-                    }
-                    if (!mbar_wait_warp(decided, n_split_units & 1, abort)) break;
-                    ++n_split_units;
-                    if (*s_last != 0 && row_ok) {
-#pragma unroll 1
-                        for (int c = 0; c < NCHUNK; ++c) {
-                            int32_t v[CH];
-#pragma unroll
-                            for (int j = 0; j < CH; ++j) {
-                                const int tok = tok_base + c * CH + j;
-                                v[j] = tok < N ? __ldcg(acc_buf + static_cast<int64_t>(tok) * M + f) : 0;
-                            }
-#pragma unroll
-                            for (int j = 0; j < CH; ++j) {
-                                const int tok = tok_base + c * CH + j;
-                                if (tok >= N) break;
-                                const int64_t o = static_cast<int64_t>(tok) * M + f;
-                                acc_buf[o] = 0;  // zero again for the next call
-                                const int32_t a = v[j] >> Cfg::ACC_SHIFT;
-                                Y[o] = dequant1(a, col_s[cg * Cfg::EPI_COLS + c * CH + j], swf, bf);
-                                if (acc_out != nullptr) acc_out[o] = a;
-                            }
-                        }
-                    }
-                }
+                if (!owner) mbar_arrive_cluster(cluster_addr(red_in, owner_rank));
             }
             mbar_arrive(scale_free);
         }
@@ -919,7 +946,8 @@ __global__ void __launch_bounds__(Cfg::NUM_THREADS, 1)
     }
 
     __syncthreads();
-    if (Cfg::PAIR) cluster_sync();  // neither CTA leaves while its peer may still signal it
+    // no CTA leaves while a peer may still signal it or read its shared memory
+    if (Cfg::PAIR || csplit) cluster_sync();
     if (warp == 1) {
         tc_fence_after_sync();
         if (Cfg::PAIR) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);

@@ -62,21 +62,20 @@ __global__ void __launch_bounds__(256) gemv_i8_kernel(const int8_t *__restrict__
             }
         }
     };
-    // (Requesting the first weights before the grid-dependency wait, to overlap
-    // the activation launch, measured slower: 7.9 against 7.2 us at M = 1,
-    // K = N = 4096, weights in HBM.)
-    pdl_wait();  // the codes and scales may come from the previous kernel
-    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         // the block's weight rows are contiguous: one bulk prefetch into L2 (TMA)
-        // puts them in flight at once, ahead of the lanes' loads (measured
-        // 4.95 -> 4.50 us at M = 1, K = N = 4096)
+        // puts them in flight at once, ahead of the lanes' loads.  The weights
+        // are not written by the previous kernel in the stream and a prefetch
+        // cannot return stale data, so it goes out before the dependency wait
+        // and overlaps the activation launch.
         const int rows = N - n0 < R ? N - n0 : R;
         const int64_t rowb = W4 ? K / 2 : K;
         asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(Wq + static_cast<int64_t>(n0) * rowb),
                      "r"(static_cast<uint32_t>(rows * rowb))
                      : "memory");
     }
+    pdl_wait();  // the codes and scales may come from the previous kernel
+    pdl_launch_dependents();
 
     int acc[R][MT];
 #pragma unroll

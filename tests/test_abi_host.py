@@ -117,8 +117,10 @@ def test_linear_workspace_bytes_adds_split_k_room(lib):
     for bits in (8, 4):
         for M, K, N in [(1, 4096, 4096), (16, 1024, 3072), (5184, 4096, 1024), (16384, 4096, 4096)]:
             assert lws(M, K, N, bits) >= ws(M, K, bits) + 2048
-    # 100 tokens against a 1024 x 4096 weight: too few feature-major tiles, room for the split sum
-    assert lws(100, 4096, 1024, 8) > ws(100, 4096, 8) + 2048
+    # few tokens: the feature-major GEMM splits K over clusters of CTAs whose
+    # partials meet in distributed shared memory, so only the counters
+    assert lws(100, 4096, 1024, 8) == ws(100, 4096, 8) + 2048
+    assert lws(16, 1024, 3072, 4) == ws(16, 1024, 4) + 2048
     # the weight-streaming kernel (one token) needs no split state beyond the counters
     assert lws(1, 4096, 4096, 8) == ws(1, 4096, 8) + 2048
     assert lws(8, 4096, 4096, 4) == ws(8, 4096, 4) + 2048
