@@ -340,7 +340,10 @@ constexpr int kMaxSplitTiles = 512;              // split-K counters in a linear
 constexpr size_t kCounterBytes = kMaxSplitTiles * 4;
 static_assert(kCounterBytes == convrot::kFuseMaxPanels * 4, "the fused linear's panel counters fill the counter area");
 constexpr int64_t kSwapMaxTokens = 128;          // feature-major up to this many tokens
-constexpr int kMinSliceSteps = 4;                // K steps of 128 in a feature-major split-K slice
+// K steps of 128 in a feature-major split-K slice (B200, CUDA-graph-timed: at
+// K = 1024 splitting in two is 0.2-0.6 us slower than whole tiles, at K = 2048
+// two slices beat four and eight, at K = 4096 four and eight tie)
+constexpr int kMinSliceSteps = 8;
 // Stream-K: the cost of the shared tiles (148 partial tiles of 128 KB stored and
 // read back, ~5 us on B200), in 128-deep steps of a 256-wide tile: int8 weights
 // / widened int4 weights (whose steps are slower).  Measured, CUDA-graph-timed,

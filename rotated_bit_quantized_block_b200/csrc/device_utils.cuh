@@ -122,12 +122,14 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 
 // ---------------------------------------------------------------- TMA
 
-// 1-D bulk copy global -> shared of `bytes` contiguous bytes (a multiple of 16;
-// both addresses 16-byte aligned), completing on `bar`.  No multicast.
-__device__ __forceinline__ void bulk_load_1d(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_addr(dst)),
-                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+// Bulk copy (TMA engine, no multicast) of `bytes` contiguous bytes -- a multiple
+// of 16, both addresses 16-byte aligned -- from this CTA's shared memory to the
+// shared memory of a CTA of the cluster.  dst and bar are shared::cluster
+// addresses in that CTA; the copied bytes are counted on its mbarrier bar
+// (complete_tx).
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "r"(smem_addr(src)), "r"(bytes), "r"(bar)
                  : "memory");
 }
 
@@ -235,6 +237,21 @@ __device__ __forceinline__ void tmem_ld_32x16(uint32_t taddr, uint32_t (&r)[16])
         : "r"(taddr));
 }
 
+// 32 lanes x 8, 4 or 2 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32x8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_32x4(uint32_t taddr, uint32_t (&r)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_32x2(uint32_t taddr, uint32_t (&r)[2]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor (sm_100 format) for a K-major operand tile
@@ -285,15 +302,23 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// The two halves of cluster_sync, for a barrier whose wait can come much later.
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // Arrive on an mbarrier given by its shared::cluster address (possibly the peer's).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
 
-// Bounded wait (every lane of the warp) for a phase completed by arrivals from
-// other CTAs of the cluster: acquire at cluster scope, so that what those CTAs'
-// threads wrote to their own shared memory before arriving (release, cluster
-// scope) is visible to this warp's distributed-shared-memory loads.
+// Bounded wait (every lane of the warp) for a phase completed by other CTAs of
+// the cluster (remote arrivals or bulk copies counted with complete_tx):
+// acquire at cluster scope, so that what they released or copied is visible
+// to this warp's loads.
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t *bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
@@ -306,35 +331,24 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t *bar, uint32_
     return done != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    bool ok = true;
-    if (!mbar_try_wait_acq_cluster(bar, parity)) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait_acq_cluster(bar, parity)) {
-            if (*abort) {
-                ok = false;
-                break;
-            }
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                atomicOr(&g_device_status, kStatusTimeout);
-                *abort = 1;
-                ok = false;
-                break;
-            }
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_acq_cluster(bar, parity)) {
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_device_status, kStatusTimeout);
+            *abort = 1;
+            return false;
         }
     }
-    return __all_sync(0xffffffffu, ok);
+    return true;
 }
 
-// 16-byte load from the shared memory of a CTA of the cluster (shared::cluster address).
-__device__ __forceinline__ uint4 ld_dsmem_v4(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xffffffffu, mbar_wait_cluster(bar, parity, abort));
 }
+
 
 // TMA load into this CTA's shared memory whose completion is counted on the
 // mbarrier of the pair's even CTA (shared::cluster address).  No multicast.

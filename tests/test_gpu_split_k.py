@@ -42,17 +42,19 @@ def sms():
 
 
 # (M, N, K, tile_n, k_splits on a 148-SM B200): every cluster size and token
-# tile width, ragged N (1000, 520) and ragged M, a split limited by K (K / 128
-# = 8 steps: two slices of 4) and a tile count too small to split (5 steps)
+# tile width, ragged N (1000, 520) and ragged M, a split limited by K (16 steps
+# of 128: two slices of 8) and shapes whose slices would be too short to split
 CASES = [
     (16, 4096, 4096, 32, 4),
-    (5, 4096, 2048, 32, 4),
+    (5, 4096, 2048, 32, 2),
+    (24, 1024, 16384, 32, 8),
     (40, 9472, 2048, 64, 2),
-    (64, 1000, 4096, 64, 8),
-    (100, 1024, 4096, 128, 8),
-    (90, 2048, 1024, 128, 2),
+    (64, 1000, 4096, 64, 4),
+    (100, 1024, 8192, 128, 8),
+    (90, 2048, 2048, 128, 2),
     (128, 2048, 8192, 128, 8),
     (33, 520, 640, 64, 1),
+    (128, 3072, 1024, 128, 1),
 ]
 
 
