@@ -476,25 +476,33 @@ def measure_workload(w, reps, stream, steps, peaks, clock_index=None, warmup=3):
     # the dominant kernel: the GEMM (the activation launch is reported under rotate_quant)
     dom_ms = sum(v["gemm_ms"] for v in per.values())
     int8_peak = 2.0 * peaks["bf16_tflops"]  # dense int8 = 2 x dense bf16 (4.5 vs 2.25 POPS nominal)
-    if all(v["plan"]["gemm_kind"] == 2 for v in per.values()):
-        # the fewest tokens: bound by reading the weights (and the activation codes)
-        moved = sum(linear_bytes(w, l) - w.M * l.K for l in w.linears)
-        achieved = moved / (dom_ms / 1e3) / 1e9
+    # the GEMM's algorithmic bytes: activation codes (one byte each), weight codes, Y and the scales
+    gemm_bytes = {l.name: linear_bytes(w, l) - w.M * l.K for l in w.linears}
+    ridge = int8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)  # int8 ops per byte where the two roofs meet
+    if ops / sum(gemm_bytes.values()) < ridge:
+        # few tokens: bound by streaming the weights (and the activation codes)
+        achieved = sum(gemm_bytes.values()) / (dom_ms / 1e3) / 1e9
+        kinds = {v["plan"]["gemm_kind"] for v in per.values()}
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "kernel": "gemv_i8 (weight-streaming, dp4a)",
-                "peak_note": f"{peaks['source']} HBM copy bandwidth"}
+                "frac": achieved / peaks["hbm_gbs"],
+                "kernel": ("gemv_i8 (weight-streaming, dp4a)" if kinds == {2} else
+                           "gemm_i8_tcgen05 feature-major (all tokens in one tile, K split over clusters)"),
+                "peak_note": f"{peaks['source']} HBM copy bandwidth; the GEMM's {ops / sum(gemm_bytes.values()):.0f} "
+                             f"int8 ops per byte lie below the ridge of {ridge:.0f}",
+                "per_linear_frac": {l.name: round(gemm_bytes[l.name] / (per[l.name]["gemm_ms"] / 1e3) / 1e9
+                                                  / peaks["hbm_gbs"], 3) for l in w.linears}}
     else:
         achieved = ops / (dom_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
                 "frac": achieved / int8_peak,
                 "kernel": "gemm_i8_tcgen05 (int8 x int8 -> int32 in TMEM, dequant epilogue)",
-                "peak_note": f"dense int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s"}
+                "peak_note": f"dense int8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s",
+                "per_linear_frac": {l.name: round(2 * w.M * l.K * l.N / (per[l.name]["gemm_ms"] / 1e3) / 1e12
+                                                  / int8_peak, 3) for l in w.linears}}
     roof.update({
         "timing": "each linear alone: CUDA graph of back-to-back launches over the rotating buffer sets, "
                   "CUDA events on the launching stream around the replay",
         "per_linear_us": {n: round(1e3 * v["gemm_ms"], 2) for n, v in per.items()},
-        "per_linear_frac": {l.name: round(2 * w.M * l.K * l.N / (per[l.name]["gemm_ms"] / 1e3) / 1e12 / int8_peak, 3)
-                            for l in w.linears},
     })
     act_total_ms = sum(v["act_ms"] for v in per.values())
     act_gbs = sum(act_bytes(w, l) for l in w.linears) / (act_total_ms / 1e3) / 1e9
@@ -634,7 +642,8 @@ def ours_arm(args, w, rank, world, local_rank):
     roofline = dict(m["roofline"])
     roofline["traffic"] = statistics.mean(traffic["gemm"].values()) if traffic["gemm"] else None
     roofline["traffic_per_linear"] = traffic["gemm"]
-    roofline["algorithmic_bytes_per_linear"] = {l.name: linear_bytes(w, l) for l in w.linears}
+    # the GEMM's own: activation codes in, weight codes, Y and the scales
+    roofline["algorithmic_bytes_per_linear"] = {l.name: linear_bytes(w, l) - w.M * l.K for l in w.linears}
     rotate_quant = dict(m["rotate_quant"])
     rotate_quant["traffic"] = statistics.mean(traffic["act"].values()) if traffic["act"] else None
     rotate_quant["traffic_per_linear"] = traffic["act"]
