@@ -236,8 +236,8 @@ cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Extra grid-stride work of the activation launch: zeroing split-K state, and
-// widening the W4A4 linear's packed weights to int8 codes.
+// Extra grid-stride work of the activation launch: zeroing the workspace's
+// counters, and widening the W4A4 linear's packed weights to int8 codes.
 struct ActExtras {
     uint4 *zero16 = nullptr;
     int64_t n_zero16 = 0;
@@ -345,8 +345,8 @@ struct GemmPlan {
     int streamk = 0;    // token-major stream-K: CTAs sharing the K steps of all tiles (0: off)
 };
 
-constexpr int kMaxSplitTiles = 512;              // split-K counters in a linear's workspace
-constexpr size_t kCounterBytes = kMaxSplitTiles * 4;
+constexpr int kCounterWords = 512;               // stream-K / fused-panel counters in a linear's workspace
+constexpr size_t kCounterBytes = kCounterWords * 4;
 static_assert(kCounterBytes == convrot::kFuseMaxPanels * 4, "the fused linear's panel counters fill the counter area");
 constexpr int64_t kSwapMaxTokens = 128;          // feature-major up to this many tokens
 // K steps of 128 in a feature-major split-K slice (B200, CUDA-graph-timed: at
@@ -835,8 +835,7 @@ convrot_status_t convrot_rotate_quant_act(const void *X, int64_t M, int64_t K, i
 
 // Workspace layout of the linears: activation codes (one byte each); at the
 // next 256-byte boundary the per-token scales; then (when the workspace is
-// large enough) kMaxSplitTiles split-K counters and the int32 M x N sum
-// buffer of a split feature-major GEMM.
+// large enough) kCounterWords counters and the stream-K partial-tile slots.
 static void workspace_parts(void *workspace, int64_t M, int64_t K, void **xq, float **xs,
                             unsigned int **counters = nullptr, int32_t **acc_buf = nullptr) {
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -864,9 +863,7 @@ static convrot_status_t check_workspace(const void *workspace, size_t workspace_
     return ok();
 }
 
-// n_features >= 0: the GEMM half's N is known, so exactly the split-K state it
-// will use is zeroed; otherwise everything after the codes and scales, up to
-// the largest split buffer a GEMM over M tokens can use.
+// n_features: the GEMM half's N where known (needed to widen weights).
 // wide: the packed int4 weights (N x K/2) to widen into the workspace (see
 // w4_prewidens), or null.
 static convrot_status_t linear_act_impl(const void *X, int64_t M, int64_t K, int block, int bits, void *workspace,

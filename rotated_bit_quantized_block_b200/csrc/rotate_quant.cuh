@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
 #pragma unroll
         for (int j = 0; j < 4; ++j) raw[j] = make_uint4(0, 0, 0, 0);
     }
-    // (while the row loads are in flight) the linear's split-K counters and sum buffer start at zero for the GEMM that follows
+    // (while the row loads are in flight) the linear's counters start at zero for the GEMM that follows
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + tid; i < n_zero16;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)
         zero16[i] = make_uint4(0u, 0u, 0u, 0u);
