@@ -589,7 +589,8 @@ convrot_status_t launch_gemv_mt(const void *Xc, const void *Wc, int64_t M, int64
                                 const float *sw, const void *bias, void *Y, int32_t *acc_out, cudaStream_t st) {
     int64_t nw = K / convrot::kGemvChunk;
     nw = nw < 1 ? 1 : (nw > 8 ? 8 : nw);
-    const int64_t grid = (N + convrot::kGemvFeatures - 1) / convrot::kGemvFeatures;
+    constexpr int R = convrot::gemv_features<MT>();
+    const int64_t grid = (N + R - 1) / R;
     launch_pdl(convrot::gemv_i8_kernel<W4, MT>, dim3(static_cast<unsigned>(grid)), dim3(static_cast<unsigned>(32 * nw)),
                0, st, static_cast<const int8_t *>(Xc), sx, static_cast<const uint8_t *>(Wc), sw,
                static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out, static_cast<int>(M),
