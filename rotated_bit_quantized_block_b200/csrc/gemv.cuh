@@ -8,7 +8,7 @@
 // Method: civarchive.com "SAM 3.1 Multiplex ConvRot" release, "Quantization
 // recipe" (W8A8 / W4A4 operations, per-row scales).  With so few tokens the
 // product is bound by reading the weights once from HBM, so the tensor core is
-// not needed: each block owns 4 or 8 output features, its warps split K into
+// not needed: each block owns 2 to 8 output features, its warps split K into
 // 512-code chunks (one 16-byte load per lane and feature), int4 weights are
 // widened in registers, the activation codes (a few KB) come through L1.
 #pragma once
@@ -17,11 +17,12 @@
 
 namespace convrot {
 
-// Output features per block: 8 for 1-2 tokens, 4 for more (measured on B200,
-// K = N = 4096, linear: 1 token 6.3 -> 5.7 us with 8, 2 tokens 7.3 -> 6.2; at 4
-// tokens 8 features were slower, 8.6 -> 9.6 us, and 16 slower everywhere).
+// Output features per block by token bound (measured on B200, K = N = 4096,
+// linear, against 4 features: 1 token 6.3 -> 5.7 us with 8, 2 tokens 7.3 ->
+// 6.2 with 8; 4 tokens 8.6 -> 8.4 with 2 and 9.6 with 8; 8 tokens best with 4;
+// 16 features slower everywhere).
 template <int MT>
-__host__ __device__ constexpr int gemv_features() { return MT <= 2 ? 8 : 4; }
+__host__ __device__ constexpr int gemv_features() { return MT <= 2 ? 8 : (MT <= 4 ? 2 : 4); }
 constexpr int kGemvChunk = 512;      // codes per warp step (32 lanes x 16)
 constexpr int kGemvMaxTokens = 16;
 
