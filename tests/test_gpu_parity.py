@@ -103,7 +103,7 @@ def test_act_bit_exact_when_butterfly_is_exact(b, bits):
     assert s[5] == 0 and np.all(q[5] == 0)
 
 
-@pytest.mark.parametrize("name,idx", [("vit_l_w8a8", 0), ("vit_l_w8a8", 3), ("vit_l_w4a4", 3), ("dit_w8a8", 2)])
+@pytest.mark.parametrize("name,idx", [("vit_l_w8a8", 0), ("vit_l_w8a8", 3), ("vit_l_w4a4", 3), ("dit_w8a8", 0), ("dit_w8a8", 2)])
 def test_act_full_size_sampled_rows(name, idx):
     w = wl.WORKLOADS[name]
     X, _, _ = wl.linear_inputs(w, idx)
