@@ -531,3 +531,48 @@ def test_w4a4_linear_widens_weights_once(M, N, K):
     rows = np.unique(np.linspace(0, M - 1, 33).astype(int))
     yr = oracle.gemm_dequant(qx[rows], sx[rows], qw, host(sw), bias)
     assert np.array_equal(y[rows].view(np.uint16), yr.view(np.uint16))
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("M", [40, 300])
+def test_degenerate_rows(M, bits):
+    """The method's degenerate inputs, on the few-token (M = 40) and token-major
+    (M = 300) GEMMs: an all-zero activation row (scale 0, codes 0, output =
+    bias), a one-hot outlier (its block rotates to equal magnitudes), a constant
+    block (rotates to a single nonzero), a row at the fp16 limit (+-65504), and
+    all-zero / one-hot weight rows.  Codes and scales meet the oracle's bar,
+    the GEMM of those codes is bit-exact, and the all-zero rows give exactly
+    the bias."""
+    K, N, b = 1024, 264, 128
+    X = wl.activations(M, K, 0.01, 30.0, seed=M + bits).astype(np.float16)
+    X[0] = 0.0
+    X[1] = 0.0
+    X[1, 5] = 1000.0
+    X[2] = 0.0
+    X[2, 128:256] = 3.0
+    X[3] = np.where(np.arange(K) % 3 == 0, -65504.0, 65504.0).astype(np.float16)
+    W = wl.weight(N, K, 0.02, seed=N + bits)
+    W[0] = 0.0
+    W[1] = 0.0
+    W[1, 700] = 0.5
+    bias = wl.bias(N, seed=bits)
+    Wq, sw = cr.convrot_quantize_weight(dev(W), b, bits, cr.CLIP_MSE)
+    _check_mse_rows(W, b, bits, unpack(host(Wq), bits), host(sw))
+    assert host(sw)[0] == 0.0 and not np.any(unpack(host(Wq), bits)[0])
+    ws = torch.empty(cr.convrot_linear_workspace_bytes(M, K, N, bits), dtype=torch.uint8, device="cuda")
+    fn = cr.convrot_linear_w8a8 if bits == 8 else cr.convrot_linear_w4a4
+    y = host(fn(dev(X), Wq, sw, b, bias=dev(bias), workspace=ws))
+    raw = host(ws)
+    qx = raw[: M * K].view(np.int8).reshape(M, K)
+    off = (M * K + 255) // 256 * 256
+    sx = raw[off: off + 4 * M].view(np.float32)
+    qx_o, sx_o = oracle.rotate_quant_act(X, b, bits)
+    assert np.allclose(sx, sx_o, rtol=1e-5, atol=0)
+    assert sx[0] == 0.0 and not np.any(qx[0])
+    assert_codes_close(qx, qx_o)
+    yr = oracle.gemm_dequant(qx, sx, unpack(host(Wq), bits), host(sw), bias)
+    assert np.array_equal(y.view(np.uint16), yr.view(np.uint16))
+    assert np.array_equal(y[0].view(np.uint16), bias.astype(np.float16).view(np.uint16))
+    # (the fp16-limit row may overflow Y to +-inf, as an fp16 linear would: the
+    # bit-exact comparison above covers it)
+    assert np.all(np.isfinite(y[:3].astype(np.float32)))
