@@ -365,7 +365,8 @@ constexpr double kStreamKOverheadSteps4 = 9.0;
 // 128 columns), so that every weight byte is read once.  Where the tiles alone
 // leave SMs idle, K is split over a cluster of 2, 4 or 8 CTAs (each slice at
 // least kMinSliceSteps steps of 128), whose partial accumulators are added
-// through distributed shared memory.  Otherwise token-major 128 x 256 tiles,
+// after shared-memory bulk copies between the cluster's CTAs.  Otherwise
+// token-major 128 x 256 tiles,
 // narrowed when narrower tiles finish in fewer rounds.  (Measured on B200 with
 // CUDA-graph launches: feature-major wins up to 128 tokens, token-major from 192.)
 GemmPlan plan_gemm(int sms, int64_t M, int64_t N, int64_t K, bool allow_split, bool w4 = false) {
