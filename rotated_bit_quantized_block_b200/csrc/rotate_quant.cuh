@@ -452,8 +452,6 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
     const int g = l >> 2, p = l & 3;
     uint8_t *xbuf = act_smem + (tid >> 2) * kXposeGroupBytes;
 
-    pdl_wait();  // X may come from, and Xq may still be read by, the previous kernel
-    pdl_launch_dependents();
     if (tid == 0 || (tid == 32 && pf_ahead > 0)) {
         // A CTA's rows are contiguous: one bulk prefetch into L2 (TMA, no
         // shared memory) puts all of their bytes in flight at once, ahead of
@@ -461,6 +459,11 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
         // GPU at once, the CTA also prefetches the rows of the CTA pf_ahead
         // places later, which runs in the next wave.  (Measured: own rows +6 %
         // to +17 %; one wave ahead another +4 % to +12 % on multi-wave grids.)
+        // It goes out before the grid-dependency wait: a prefetch is only a
+        // hint and L2 is the point of coherence, so rows that the previous
+        // kernel is still writing are read correctly by the loads after the
+        // wait, and CTAs that become resident during the previous kernel's
+        // last partial round of tiles overlap their reads with it.
         const int64_t cta = static_cast<int64_t>(blockIdx.x) + (tid == 0 ? 0 : pf_ahead);
         const int64_t r0 = cta * rows;
         if (r0 < M) {
@@ -470,6 +473,8 @@ __global__ void __launch_bounds__(1024) act_rotate_quant_kernel(const __half *__
                          : "memory");
         }
     }
+    pdl_wait();  // X may come from, and Xq may still be read by, the previous kernel
+    pdl_launch_dependents();
     uint4 raw[4];
     if (active) {
         const __half *src = X + row * K + 128 * g + 8 * p;
