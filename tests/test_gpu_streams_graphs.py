@@ -5,10 +5,12 @@ dependent launch, and all its state lives in the caller's workspace, so
 (a) linears of different shapes and plans (weight-streaming, feature-major
 split K over clusters, token-major tiles, CTA pairs, W4A4 with widened
 weights) running at the same time on independent streams and workspaces must
-each give exactly what they give alone, and (b) a chain of such linears
+each give exactly what they give alone, (b) a chain of such linears
 captured once in a CUDA graph must give, on every replay, exactly what the
-same chain gives when launched eagerly.  Integer sums are exact and the
-epilogue rounds identically, so the comparisons are bit for bit.
+same chain gives when launched eagerly, and (c) a linear fed the previous
+linear's output must quantize the finished rows although its launch may
+start during the previous GEMM.  Integer sums are exact and the epilogue
+rounds identically, so the comparisons are bit for bit.
 Source: civarchive "SAM 3.1 Multiplex ConvRot" release, "Quantization recipe"
 (online activation quantization, integer GEMM, per-row dequantization).
 """
@@ -95,4 +97,60 @@ def test_chain_of_linears_in_one_graph():
         torch.cuda.synchronize()
         for it, r in zip(items, ref):
             assert torch.equal(it["Y"].view(torch.int16), r.view(torch.int16))
+    del g
+
+
+# (M, K, N1, N2, bits): an MLP pair at ViT-L width (token-major GEMMs), few
+# tokens (feature-major clusters, the weight-streaming kernel), int4 weights
+CHAINS = [(5184, 1024, 4096, 1024, 8), (5184, 1024, 4096, 1024, 4), (16, 4096, 4096, 4096, 8),
+          (1, 4096, 4096, 4096, 8), (300, 1024, 2048, 1024, 4)]
+
+
+@pytest.mark.parametrize("shared_ws", [False, True])
+@pytest.mark.parametrize("M,K,N1,N2,bits", CHAINS)
+def test_linear_consumes_the_previous_linears_output(M, K, N1, N2, bits, shared_ws):
+    """The second linear's activation launch may become resident, and start
+    fetching its rows, while the first linear's GEMM is still writing them;
+    what it quantizes must be the finished rows.  Back-to-back launches, eager
+    and replayed from a CUDA graph, equal the same two calls with a device
+    synchronisation between them, bit for bit (also when both linears share
+    one workspace, so the second's codes overwrite those the first GEMM read)."""
+    first = make(M, K, N1, bits, seed=M + 1)
+    second = make(M, N1, N2, bits, seed=M + 2)
+    second["X"] = first["Y"]
+    if shared_ws:
+        n = max(first["ws"].numel(), second["ws"].numel())
+        first["ws"] = second["ws"] = torch.empty(n, dtype=torch.uint8, device="cuda")
+    run(first)
+    torch.cuda.synchronize()
+    run(second)
+    torch.cuda.synchronize()
+    ref1, ref2 = first["Y"].clone(), second["Y"].clone()
+    assert torch.isfinite(ref2.float()).all()
+
+    def zero():
+        first["Y"].fill_(0)
+        second["Y"].fill_(0)
+        torch.cuda.synchronize()
+
+    def check():
+        torch.cuda.synchronize()
+        assert torch.equal(first["Y"].view(torch.int16), ref1.view(torch.int16))
+        assert torch.equal(second["Y"].view(torch.int16), ref2.view(torch.int16))
+
+    st = torch.cuda.Stream()
+    for _ in range(3):
+        zero()
+        with torch.cuda.stream(st):
+            run(first, st)
+            run(second, st)
+        check()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        run(first, st)
+        run(second, st)
+    for _ in range(2):
+        zero()
+        g.replay()
+        check()
     del g
