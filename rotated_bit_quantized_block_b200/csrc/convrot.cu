@@ -583,30 +583,49 @@ convrot_status_t launch_gemm_cfg(DeviceInfo *info, int dev, const void *Xc, cons
     return launch_status("gemm_i8_tcgen05");
 }
 
-// Weight-streaming GEMM for M <= 16 tokens (int8 activation codes; W4 = packed
-// int4 weights): blocks of 4 output features, warps splitting K.
-template <bool W4, int MT>
+// Weight-streaming GEMM for the fewest tokens (int8 activation codes; W4 =
+// packed int4 weights): blocks of R output features, at most `max_warps`
+// warps splitting K in 512-code chunks.
+template <bool W4, int MT, int R>
 convrot_status_t launch_gemv_mt(const void *Xc, const void *Wc, int64_t M, int64_t N, int64_t K, const float *sx,
-                                const float *sw, const void *bias, void *Y, int32_t *acc_out, cudaStream_t st) {
+                                const float *sw, const void *bias, void *Y, int32_t *acc_out, cudaStream_t st,
+                                int64_t max_warps) {
     int64_t nw = K / convrot::kGemvChunk;
-    nw = nw < 1 ? 1 : (nw > 8 ? 8 : nw);
-    constexpr int R = convrot::gemv_features<MT>();
+    nw = nw < 1 ? 1 : (nw > max_warps ? max_warps : nw);
     const int64_t grid = (N + R - 1) / R;
-    launch_pdl(convrot::gemv_i8_kernel<W4, MT>, dim3(static_cast<unsigned>(grid)), dim3(static_cast<unsigned>(32 * nw)),
-               0, st, static_cast<const int8_t *>(Xc), sx, static_cast<const uint8_t *>(Wc), sw,
-               static_cast<const __half *>(bias), static_cast<__half *>(Y), acc_out, static_cast<int>(M),
-               static_cast<int>(N), static_cast<int>(K));
+    launch_pdl(convrot::gemv_i8_kernel<W4, MT, R>, dim3(static_cast<unsigned>(grid)),
+               dim3(static_cast<unsigned>(32 * nw)), 0, st, static_cast<const int8_t *>(Xc), sx,
+               static_cast<const uint8_t *>(Wc), sw, static_cast<const __half *>(bias), static_cast<__half *>(Y),
+               acc_out, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K));
     return launch_status("gemv_i8");
 }
 
+// Features per block and warps per block (B200, CUDA graphs, weights beyond
+// L2, the linear / its GEMM alone, us):
+//  * int8 weights, 1-2 tokens: 4 features and at most 4 warps where the grid
+//    is wide and K moderate (K = N = 4096: 1 token 6.37 / 4.40 -> 5.84 /
+//    4.35, 2 tokens 6.77 -> 6.42 linear; 1 x 1024 -> 3072 3.50 -> 3.44),
+//    otherwise 8 and 8 (1 x 4096 -> 1024: 4.00 against 4.18 with 4 and 4;
+//    1 x 16384 -> 4096 GEMM alone 12.2 against 14.5);
+//  * int4 weights, 1-2 tokens: 8 and 8 (half the bytes per lane load; with 4
+//    and 4 1 token 5.33 -> 5.40, 2 tokens 5.90 -> 6.18);
+//  * 3-8 tokens: 2 (up to 4 tokens) or 4 features and at most 4 warps (int8
+//    3 / 4 tokens 8.11 / 8.62 -> 7.37 / 7.88, int4 4 / 8 tokens 8.05 / 13.1
+//    -> 7.17 / 11.45 against 8 warps).
 template <bool W4>
 convrot_status_t launch_gemv(const void *Xc, const void *Wc, int64_t M, int64_t N, int64_t K, const float *sx,
                              const float *sw, const void *bias, void *Y, int32_t *acc_out, cudaStream_t st) {
-    if (M <= 1) return launch_gemv_mt<W4, 1>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
-    if (M <= 2) return launch_gemv_mt<W4, 2>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
-    if (M <= 4) return launch_gemv_mt<W4, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
-    if (M <= 8) return launch_gemv_mt<W4, 8>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
-    return launch_gemv_mt<W4, 16>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st);
+    if (M <= 2) {
+        if (!W4 && N >= 2048 && K <= 8192) {
+            if (M <= 1) return launch_gemv_mt<W4, 1, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
+            return launch_gemv_mt<W4, 2, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
+        }
+        if (M <= 1) return launch_gemv_mt<W4, 1, 8>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
+        return launch_gemv_mt<W4, 2, 8>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
+    }
+    if (M <= 4) return launch_gemv_mt<W4, 4, 2>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
+    if (M <= 8) return launch_gemv_mt<W4, 8, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
+    return CONVROT_ERR_UNSUPPORTED;  // the planner hands at most 8 tokens to this kernel
 }
 
 // X4 / W4: activation / weight codes packed int4.

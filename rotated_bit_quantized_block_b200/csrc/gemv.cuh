@@ -1,6 +1,6 @@
 // gemv.cuh -- the integer GEMM with its dequantizing epilogue for a handful of
-// tokens (the plan uses it up to 4 tokens with int8 weights, 8 with int4; the
-// kernel accepts up to 16), as a weight-streaming kernel.
+// tokens (the plan uses it up to 4 tokens with int8 weights, 8 with int4), as
+// a weight-streaming kernel.
 //
 //   acc[m,n] = sum_k qx[m,k] * qw[n,k]            (exact int32, dp4a)
 //   Y[m,n]   = fp16( fma( fp32(float(acc) * s_x[m]), s_w[n], bias[n] ) )
@@ -8,7 +8,7 @@
 // Method: civarchive.com "SAM 3.1 Multiplex ConvRot" release, "Quantization
 // recipe" (W8A8 / W4A4 operations, per-row scales).  With so few tokens the
 // product is bound by reading the weights once from HBM, so the tensor core is
-// not needed: each block owns 2 to 8 output features, its warps split K into
+// not needed: each block owns 2, 4 or 8 output features, its warps split K into
 // 512-code chunks (one 16-byte load per lane and feature), int4 weights are
 // widened in registers, the activation codes (a few KB) come through L1.
 #pragma once
@@ -17,14 +17,7 @@
 
 namespace convrot {
 
-// Output features per block by token bound (measured on B200, K = N = 4096,
-// linear, against 4 features: 1 token 6.3 -> 5.7 us with 8, 2 tokens 7.3 ->
-// 6.2 with 8; 4 tokens 8.6 -> 8.4 with 2 and 9.6 with 8; 8 tokens best with 4;
-// 16 features slower everywhere).
-template <int MT>
-__host__ __device__ constexpr int gemv_features() { return MT <= 2 ? 8 : (MT <= 4 ? 2 : 4); }
 constexpr int kGemvChunk = 512;      // codes per warp step (32 lanes x 16)
-constexpr int kGemvMaxTokens = 16;
 
 __device__ __forceinline__ uint2 ld_stream_v2(const void *p) {
     uint2 v;
@@ -42,14 +35,13 @@ __device__ __forceinline__ uint4 gemv_widen_int4x16(uint2 p) {
 }
 
 // Xq: M x K int8 codes; Wq: N x K int8 (W4 = false) or N x K/2 packed int4
-// (W4 = true); MT >= M is the compile-time token bound.  Block: nw warps
-// (blockDim.x = 32 * nw), grid: ceil(N / gemv_features<MT>()) blocks.
-template <bool W4, int MT>
+// (W4 = true); MT >= M is the compile-time token bound, R the output features
+// per block.  Block: nw <= 8 warps (blockDim.x = 32 * nw), grid: ceil(N / R).
+template <bool W4, int MT, int R>
 __global__ void __launch_bounds__(256) gemv_i8_kernel(const int8_t *__restrict__ Xq, const float *__restrict__ sx,
                                                       const uint8_t *__restrict__ Wq, const float *__restrict__ sw,
                                                       const __half *__restrict__ bias, __half *__restrict__ Y,
                                                       int32_t *__restrict__ acc_out, int M, int N, int K) {
-    constexpr int R = gemv_features<MT>();
     constexpr int SHIFT = W4 ? 4 : 0;
     __shared__ int s_acc[8][R * MT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
