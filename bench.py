@@ -115,56 +115,160 @@ def load_traffic(workload: str):
 
 # ------------------------------------------------------------------------------------------ clocks
 
-class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+# A separate process polls NVML (the library nvidia-smi reads; nothing is set)
+# every millisecond, so that samples fall inside a timed region of a few
+# milliseconds.  Each line: monotonic time, SM MHz, max SM MHz, power W, and the
+# flags hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap.
+_NVML_POLLER = r"""
+import sys, time, pynvml
+dev, out, period = sys.argv[1], sys.argv[2], float(sys.argv[3])
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByUUID(dev) if dev.startswith("GPU-") else pynvml.nvmlDeviceGetHandleByIndex(int(dev))
+mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+        pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap)
+with open(out, "w", buffering=1) as f:
+    f.write("ready\n")
+    while True:
+        t = time.monotonic()
+        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+        f.write("%.6f,%d,%d,%.1f,%s\n" % (t, sm, mx, pw, ",".join("1" if rs & b else "0" for b in bits)))
+        time.sleep(period)
+"""
+_REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index: int):
-        self.index = index
+
+def summarize_clock_samples(lines, t0, t1):
+    """Clock record of the timed region [t0, t1] (host monotonic seconds) from
+    the poller's lines: the samples inside it, else the three nearest to it."""
+    rows = []
+    for line in lines:
+        parts = line.strip().split(",")
+        if len(parts) != 8:
+            continue
+        try:
+            rows.append((float(parts[0]), float(parts[1]), float(parts[2]), float(parts[3]),
+                         [p == "1" for p in parts[4:8]]))
+        except ValueError:
+            continue
+    if not rows:
+        return None
+    inside = [r for r in rows if t0 <= r[0] <= t1]
+    window = "inside the timed region"
+    if not inside:
+        mid = 0.5 * (t0 + t1)
+        inside = sorted(rows, key=lambda r: abs(r[0] - mid))[:3]
+        window = "nearest to the timed region"
+    return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+            "reasons": sorted({n for r in inside for n, on in zip(_REASONS, r[4]) if on}),
+            "samples": len(inside), "window": window, "window_ms": round(1e3 * (t1 - t0), 3),
+            "power_w_max": max(r[3] for r in inside), "source": "NVML, polled every 1 ms"}
+
+
+def nvml_device_id(device) -> str:
+    """The device's NVML id: its UUID ("GPU-" and 8-4-4-4-12 hex digits, which
+    does not depend on CUDA_VISIBLE_DEVICES), else its CUDA index."""
+    try:
+        h = bytes(int(x) & 0xFF for x in torch.cuda.get_device_properties(device).uuid.bytes).hex()
+        if len(h) == 32:
+            return f"GPU-{h[:8]}-{h[8:12]}-{h[12:16]}-{h[16:20]}-{h[20:]}"
+    except Exception:  # noqa: BLE001 -- properties without a UUID
+        pass
+    return str(device.index)
+
+
+class ClockSampler:
+    """Samples the SM clock and throttle reasons during the timed region: a
+    separate process polls NVML every millisecond (nvidia-smi at 100 ms where
+    the Python NVML bindings are missing); ``mark_start`` / ``mark_end`` bracket
+    the region on the host's monotonic clock."""
+    SMI_QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_id: str):
+        self.dev_id = dev_id
         self.proc = None
+        self.smi = False
+        self.smi_out = None
+        self.t0 = self.t1 = None
         self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.out.close()
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.out, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
+            self.proc = subprocess.Popen([sys.executable, "-c", _NVML_POLLER, self.dev_id, self.out.name, "0.001"],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            ready, deadline = False, time.monotonic() + 20.0
+            while not ready and time.monotonic() < deadline and self.proc.poll() is None:
+                with open(self.out.name) as f:
+                    ready = f.read(6) == "ready\n"
+                if not ready:
+                    time.sleep(0.01)
+            if not ready:
+                raise OSError("the NVML poller did not start")
         except (FileNotFoundError, OSError):
-            self.proc = None
+            self.stop()
+            self.smi = True
+            try:
+                self.smi_out = open(self.out.name, "w")
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", self.dev_id, f"--query-gpu={self.SMI_QUERY}",
+                                              "--format=csv,noheader,nounits", "-lms", "100"],
+                                             stdout=self.smi_out, stderr=subprocess.DEVNULL)
+                time.sleep(0.3)
+            except (FileNotFoundError, OSError):
+                self.proc = None
+        time.sleep(0.02)  # a few samples before the region
         return self
 
-    def __exit__(self, *exc):
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
+
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+            self.proc = None
+        if self.smi_out is not None:
+            self.smi_out.close()
+            self.smi_out = None
+
+    def __exit__(self, *exc):
+        time.sleep(0.02)  # samples after the region
+        self.stop()
 
     def summary(self):
-        if self.proc is None:
+        try:
+            with open(self.out.name) as f:
+                lines = f.readlines()
+            os.unlink(self.out.name)
+        except OSError:
             return None
-        self.out.flush()
-        rows = []
-        with open(self.out.name) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) == 9:
-                    rows.append(parts)
-        os.unlink(self.out.name)
-        if not rows:
+        if self.t0 is None or self.t1 is None:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
+        if not self.smi:
+            return summarize_clock_samples(lines, self.t0, self.t1)
+        # nvidia-smi fallback: no timestamps, the samples around the region
+        rows = [[p.strip() for p in line.split(",")] for line in lines]
+        rows = [r for r in rows if len(r) == 7]
+        num = lambda v: float(v) if v.replace(".", "").isdigit() else None  # noqa: E731
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted({n for r in rows for n, v in zip(_REASONS, r[3:7]) if v.lower() == "active"}),
+                "samples": len(rows), "window": "around the timed region", "window_ms": round(1e3 * (self.t1 - self.t0), 3),
+                "power_w_max": max((num(r[2]) for r in rows if num(r[2]) is not None), default=None),
+                "source": "nvidia-smi, every 100 ms"}
 
 
 # ------------------------------------------------------------------------------------------ workload
@@ -427,10 +531,12 @@ def measure_workload(w, reps, stream, steps, peaks, clock_index=None, warmup=3):
         torch.cuda.synchronize()
         if clock_index is not None:
             with ClockSampler(clock_index) as clk:
+                clk.mark_start()
                 start.record(stream)
                 g.replay()
                 end.record(stream)
                 torch.cuda.synchronize()
+                clk.mark_end()
             clocks = clk.summary()
         else:
             start.record(stream)
@@ -606,7 +712,8 @@ def ours_arm(args, w, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    m = measure_workload(w, reps, stream, args.steps, peaks, clock_index=device.index, warmup=args.warmup)
+    m = measure_workload(w, reps, stream, args.steps, peaks, clock_index=nvml_device_id(device),
+                         warmup=args.warmup)
     if world > 1:
         torch.distributed.barrier()
     elapsed_ms = max_over_ranks(m["elapsed_ms"], world, device)
