@@ -605,8 +605,11 @@ convrot_status_t launch_gemv_mt(const void *Xc, const void *Wc, int64_t M, int64
 //  * int8 weights, 1-2 tokens: 4 features and at most 4 warps where the grid
 //    is wide and K moderate (K = N = 4096: 1 token 6.37 / 4.40 -> 5.84 /
 //    4.35, 2 tokens 6.77 -> 6.42 linear; 1 x 1024 -> 3072 3.50 -> 3.44),
-//    otherwise 8 and 8 (1 x 4096 -> 1024: 4.00 against 4.18 with 4 and 4;
-//    1 x 16384 -> 4096 GEMM alone 12.2 against 14.5);
+//    and 2 features for one token from K = 4096 (K = N = 4096: 6.00 / 4.33
+//    -> 5.83 / 4.10; 1 x 8192 -> 4096 GEMM alone 7.5 -> 6.8; at K = 1024
+//    slower, 3.49 -> 3.78), otherwise 8 and 8 (1 x 4096 -> 1024: 4.00
+//    against 4.18 with 4 and 4; 1 x 16384 -> 4096 GEMM alone 12.2 against
+//    14.5);
 //  * int4 weights, 1-2 tokens: 8 and 8 (half the bytes per lane load; with 4
 //    and 4 1 token 5.33 -> 5.40, 2 tokens 5.90 -> 6.18);
 //  * 3-8 tokens: 2 (up to 4 tokens) or 4 features and at most 4 warps (int8
@@ -617,6 +620,8 @@ convrot_status_t launch_gemv(const void *Xc, const void *Wc, int64_t M, int64_t 
                              const float *sw, const void *bias, void *Y, int32_t *acc_out, cudaStream_t st) {
     if (M <= 2) {
         if (!W4 && N >= 2048 && K <= 8192) {
+            if (M <= 1 && K >= 4096)
+                return launch_gemv_mt<W4, 1, 2>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
             if (M <= 1) return launch_gemv_mt<W4, 1, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
             return launch_gemv_mt<W4, 2, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
         }
