@@ -612,9 +612,12 @@ convrot_status_t launch_gemv_mt(const void *Xc, const void *Wc, int64_t M, int64
 //    14.5);
 //  * int4 weights, 1-2 tokens: 8 and 8 (half the bytes per lane load; with 4
 //    and 4 1 token 5.33 -> 5.40, 2 tokens 5.90 -> 6.18);
-//  * 3-8 tokens: 2 (up to 4 tokens) or 4 features and at most 4 warps (int8
-//    3 / 4 tokens 8.11 / 8.62 -> 7.37 / 7.88, int4 4 / 8 tokens 8.05 / 13.1
-//    -> 7.17 / 11.45 against 8 warps).
+//  * 3-8 tokens: at most 4 warps (int8 3 / 4 tokens 8.11 / 8.62 -> 7.37 /
+//    7.88, int4 4 / 8 tokens 8.05 / 13.1 -> 7.17 / 11.45 against 8 warps),
+//    2 features up to 4 tokens (1 feature: 4 x 4096 -> 4096 7.99 -> 9.92);
+//    5-8 tokens 4 features from N = 4096, else 2 (int4 8 x 1024 -> 3072
+//    6.19 -> 5.82, 6 x 4096 -> 1024 8.51 -> 7.50; 8 x 4096 -> 4096 11.46
+//    with 4, 14.2 with 2).
 template <bool W4>
 convrot_status_t launch_gemv(const void *Xc, const void *Wc, int64_t M, int64_t N, int64_t K, const float *sx,
                              const float *sw, const void *bias, void *Y, int32_t *acc_out, cudaStream_t st) {
@@ -629,7 +632,8 @@ convrot_status_t launch_gemv(const void *Xc, const void *Wc, int64_t M, int64_t 
         return launch_gemv_mt<W4, 2, 8>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
     }
     if (M <= 4) return launch_gemv_mt<W4, 4, 2>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
-    if (M <= 8) return launch_gemv_mt<W4, 8, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
+    if (M <= 8 && N >= 4096) return launch_gemv_mt<W4, 8, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
+    if (M <= 8) return launch_gemv_mt<W4, 8, 2>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
     return CONVROT_ERR_UNSUPPORTED;  // the planner hands at most 8 tokens to this kernel
 }
 

@@ -454,13 +454,13 @@ def test_linear_with_tensorwise_weights(bits):
 
 @pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (1, 2056, 8192), (1, 3072, 1024), (2, 2056, 8192),
-                                   (1, 1000, 16384), (2, 1032, 2048),
+                                   (1, 1000, 16384), (2, 1032, 2048), (6, 4096, 1024), (5, 1024, 4096),
                                    (3, 1000, 1024), (4, 2056, 640), (8, 3072, 128), (7, 520, 8192)])
 def test_weight_streaming_gemm_bit_exact(M, N, K, bits):
     """For the fewest tokens the linear's GEMM streams the weights (dp4a, exact
     int32): bit-exact against the oracle's GEMM of the workspace's codes, for
     every block width (2, 4 and 8 features for 1-2 tokens, by N and K; 2 for
-    3-4 tokens; 4 for 5-8) and warp count (K from 128 to 16384)."""
+    3-4 tokens; 2 and 4 for 5-8, by N) and warp count (K from 128 to 16384)."""
     X = wl.activations(M, K, 0.01, 30.0, seed=M + K)
     W = wl.weight(N, K, 0.02, seed=N)
     bias = wl.bias(N, seed=4)
