@@ -607,11 +607,15 @@ convrot_status_t launch_gemv_mt(const void *Xc, const void *Wc, int64_t M, int64
 //    4.35, 2 tokens 6.77 -> 6.42 linear; 1 x 1024 -> 3072 3.50 -> 3.44),
 //    and 2 features for one token from K = 4096 (K = N = 4096: 6.00 / 4.33
 //    -> 5.83 / 4.10; 1 x 8192 -> 4096 GEMM alone 7.5 -> 6.8; at K = 1024
-//    slower, 3.49 -> 3.78), otherwise 8 and 8 (1 x 4096 -> 1024: 4.00
-//    against 4.18 with 4 and 4; 1 x 16384 -> 4096 GEMM alone 12.2 against
-//    14.5);
-//  * int4 weights, 1-2 tokens: 8 and 8 (half the bytes per lane load; with 4
-//    and 4 1 token 5.33 -> 5.40, 2 tokens 5.90 -> 6.18);
+//    slower, 3.49 -> 3.78);
+//  * the other 1-2 token cases (int4 weights among them): at most 8 warps
+//    (1 x 16384 -> 4096 GEMM alone 12.2 against 14.5 with 4; int4 K = N =
+//    4096 5.33 against 5.98) and 8 features, halved down to 2 while the grid
+//    would hold fewer than 48 K threads, since the weight loads' latency is
+//    covered by threads, not by bytes per thread (int8 1 x 4096 -> 1024
+//    3.93 -> 3.77 with 4, 1 x 2048 -> 1024 3.48 -> 3.41 with 2; int4 1 x
+//    4096 -> 1024 4.26 -> 3.88 and 1 x 1024 -> 3072 3.70 -> 3.48 with 4;
+//    int4 K = N = 4096 stays at 8: 5.28, 6.38 with 4);
 //  * 3-8 tokens: at most 4 warps (int8 3 / 4 tokens 8.11 / 8.62 -> 7.37 /
 //    7.88, int4 4 / 8 tokens 8.05 / 13.1 -> 7.17 / 11.45 against 8 warps),
 //    2 features up to 4 tokens (1 feature: 4 x 4096 -> 4096 7.99 -> 9.92);
@@ -628,8 +632,18 @@ convrot_status_t launch_gemv(const void *Xc, const void *Wc, int64_t M, int64_t 
             if (M <= 1) return launch_gemv_mt<W4, 1, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
             return launch_gemv_mt<W4, 2, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
         }
-        if (M <= 1) return launch_gemv_mt<W4, 1, 8>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
-        return launch_gemv_mt<W4, 2, 8>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
+        int64_t nw = K / convrot::kGemvChunk;
+        nw = nw < 1 ? 1 : (nw > 8 ? 8 : nw);
+        int r = 8;
+        while (r > 2 && (N + r - 1) / r * nw * 32 < 48 * 1024) r /= 2;
+        if (M <= 1) {
+            if (r == 8) return launch_gemv_mt<W4, 1, 8>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
+            if (r == 4) return launch_gemv_mt<W4, 1, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
+            return launch_gemv_mt<W4, 1, 2>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
+        }
+        if (r == 8) return launch_gemv_mt<W4, 2, 8>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
+        if (r == 4) return launch_gemv_mt<W4, 2, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
+        return launch_gemv_mt<W4, 2, 2>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 8);
     }
     if (M <= 4) return launch_gemv_mt<W4, 4, 2>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
     if (M <= 8 && N >= 4096) return launch_gemv_mt<W4, 8, 4>(Xc, Wc, M, N, K, sx, sw, bias, Y, acc_out, st, 4);
