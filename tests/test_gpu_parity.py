@@ -455,7 +455,8 @@ def test_linear_with_tensorwise_weights(bits):
 @pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (1, 2056, 8192), (1, 3072, 1024), (2, 2056, 8192),
                                    (1, 1000, 16384), (2, 1032, 2048), (6, 4096, 1024), (5, 1024, 4096),
-                                   (1, 1024, 4096), (2, 1024, 1024), (1, 1024, 2048),
+                                   (1, 1024, 4096), (2, 1024, 1024), (1, 1024, 2048), (1, 4096, 16384),
+                                   (2, 2056, 16384), (2, 1024, 4096),
                                    (3, 1000, 1024), (4, 2056, 640), (8, 3072, 128), (7, 520, 8192)])
 def test_weight_streaming_gemm_bit_exact(M, N, K, bits):
     """For the fewest tokens the linear's GEMM streams the weights (dp4a, exact
